@@ -1,0 +1,122 @@
+"""Small seeded cases for oracle pins and GPU parity (test-side only)."""
+import math
+
+import numpy as np
+
+from tree_verification_jsv_b200 import synth
+
+
+def bf16(x):
+    return synth.f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def f64(bits):
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def small_case(parents, prefixes, Hq=4, Hkv=2, D=16, seed=0, identity=False, q_scale=1.0):
+    """Arbitrary trees (request-local parent arrays) over paged caches with
+    N(0,1)/sqrt(D) bf16 values drawn from a seeded generator."""
+    rng = np.random.default_rng(seed)
+    nodes = [len(p) for p in parents]
+    offs = np.zeros(len(parents) + 1, dtype=np.int32)
+    offs[1:] = np.cumsum(nodes)
+    table, num_pages = synth.make_paging(seed, prefixes, nodes, identity=identity)
+    T = int(offs[-1])
+    s = 1.0 / math.sqrt(D)
+    return dict(
+        Hq=Hq, Hkv=Hkv, D=D,
+        page_table=table, num_pages=num_pages,
+        prefix_len=np.asarray(prefixes, dtype=np.int32),
+        node_offsets=offs,
+        parent=np.concatenate([np.asarray(p, dtype=np.int32) for p in parents]),
+        q=bf16(rng.standard_normal((T, Hq, D)) * s * q_scale),
+        k_cache=bf16(rng.standard_normal((num_pages, 16, Hkv, D)) * s),
+        v_cache=bf16(rng.standard_normal((num_pages, 16, Hkv, D)) * s),
+        scale=float(np.float32(1.0 / math.sqrt(D))),
+    )
+
+
+def logical_rows(cache_bits, page_table, b, n_slots):
+    """[n_slots, Hkv, D] fp64 rows of request b's logical sequence."""
+    flat = cache_bits.reshape(-1, cache_bits.shape[2], cache_bits.shape[3])
+    s = np.arange(n_slots)
+    phys = page_table[b, s // 16].astype(np.int64) * 16 + s % 16
+    return f64(flat[phys])
+
+
+def ancestor_matrix(parent):
+    """A[i, j] = True iff j is i or an ancestor of i (topological input)."""
+    n = len(parent)
+    A = np.zeros((n, n), dtype=bool)
+    for i in range(n):
+        if parent[i] >= 0:
+            A[i] = A[parent[i]]
+        A[i, i] = True
+    return A
+
+
+def dense_tree_attention(case):
+    """Independent reference: numpy dense attention over each request's
+    logical sequence with an explicit [N, P+N] visibility mask."""
+    Hq, Hkv, D = case["Hq"], case["Hkv"], case["D"]
+    G = Hq // Hkv
+    offs = case["node_offsets"]
+    out = np.zeros((int(offs[-1]), Hq, D))
+    for b in range(len(offs) - 1):
+        s0, s1 = int(offs[b]), int(offs[b + 1])
+        n = s1 - s0
+        P = int(case["prefix_len"][b])
+        K = logical_rows(case["k_cache"], case["page_table"], b, P + n)
+        V = logical_rows(case["v_cache"], case["page_table"], b, P + n)
+        mask = np.zeros((n, P + n), dtype=bool)
+        mask[:, :P] = True
+        mask[:, P:] = ancestor_matrix(case["parent"][s0:s1])
+        for h in range(Hq):
+            g = h // G
+            Q = f64(case["q"][s0:s1, h])
+            S = case["scale"] * (Q @ K[:, g].T)
+            S[~mask] = -np.inf
+            S -= S.max(axis=1, keepdims=True)
+            Pm = np.exp(S)
+            Pm /= Pm.sum(axis=1, keepdims=True)
+            out[s0:s1, h] = Pm @ V[:, g]
+    return out
+
+
+def run_oracle_attention(case, rows=None):
+    import oracle
+    return oracle.tree_attention(Hq=case["Hq"], Hkv=case["Hkv"], D=case["D"],
+                                 page_table=case["page_table"], prefix_len=case["prefix_len"],
+                                 node_offsets=case["node_offsets"], parent=case["parent"],
+                                 q=case["q"], k_cache=case["k_cache"], v_cache=case["v_cache"],
+                                 scale=case["scale"], rows=rows)
+
+
+def golden(name):
+    import json
+    from pathlib import Path
+    return json.loads((Path(__file__).resolve().parent / "golden" / f"lmhead_{name}.json").read_text())
+
+
+def golden_workload(name, **kw):
+    """Workload with the certified hidden-row redraws and planted tokens."""
+    g = golden(name)
+    wl = synth.make_workload(name, redraws={int(k): v for k, v in g["redraws"].items()}, **kw)
+    tokens = np.asarray(g["tokens"], dtype=np.int32)
+    return wl, tokens, np.asarray(g["argmax"], dtype=np.int64)
+
+
+def attention_close(got, want, what=""):
+    """Tolerance: |g - o| <= 2e-2 + 1e-2 |o| elementwise (bf16 output, fp32
+    accumulation), plus a tight check |g - o| <= 1e-2 |o| + 1e-3 max|o| so a
+    near-zero or partial result cannot hide inside the absolute term."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    err = np.abs(got - want)
+    assert np.all(err <= 2e-2 + 1e-2 * np.abs(want)), f"{what}: max abs err {err.max()}"
+    tight = 1e-2 * np.abs(want) + 1e-3 * np.abs(want).max()
+    bad = err > tight
+    assert not bad.any(), (f"{what}: {bad.sum()} elems beyond tight bound, max err {err.max()}, "
+                           f"max|o| {np.abs(want).max()}")
+    return float(err.max())
