@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the one-forward tree verification step; prints ONE JSON line.
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+tree attention, LM head + argmax, accept walk and KV compaction, i.e. the
+four calls of ``include/jsv.h`` on one stream.  Inputs are resident in HBM
+when the timed region starts; L2 is flushed (a 512 MB write) before every
+timed step, outside its events.  Step and per-call times come from CUDA
+events on the launching stream.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Multi-GPU: the path does not shard inside one step (replicas only), so
+under torchrun every rank runs its own replica of the workload; the value is
+all ranks' nodes divided by the slowest rank's time (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from datetime import timedelta
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "verified tree nodes/sec & verify-step latency; achieved HBM GB/s vs roofline"
+
+DESCRIPTION = {
+    "tiny": "tiny: 1 request, 2 q heads / 1 kv head, head_dim 64, hidden 256, vocab 1024, prefix 128, 16-node tree",
+    "8b_64": "Qwen3-8B-shaped single request: 32q/8kv heads, head_dim 128, hidden 4096, vocab 151936, prefix 2048, 64-node tree (depth 8, top-4)",
+    "8b_256": "Qwen3-8B-shaped long context: 32q/8kv, head_dim 128, hidden 4096, vocab 151936, prefix 16384, 256-node tree (depth 16, top-8)",
+    "ragged16": "ragged batch of 16, Qwen3-8B shapes: prefixes U[512,8192], 32-128-node trees of depth 4-12",
+    "30b_512x4": "Qwen3-30B-A3B-shaped: 32q/4kv, head_dim 128, hidden 2048, vocab 151936, batch 4, prefix 32768, 512-node trees (depth 16, top-8)",
+}
+
+CLOCK_FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+                "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["jsv", "reference"], default="jsv")
+    ap.add_argument("--workload", default="8b_64", choices=list(DESCRIPTION))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def golden(name):
+    return json.loads((ROOT / "tests" / "golden" / f"lmhead_{name}.json").read_text())
+
+
+def load_workload(name):
+    from tree_verification_jsv_b200 import synth
+    g = golden(name)
+    wl = synth.make_workload(name, redraws={int(k): v for k, v in g["redraws"].items()})
+    return wl, np.asarray(g["tokens"], dtype=np.int32), g
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def workload_model(wl):
+    """Algorithmic bytes / flops of each call and of the step."""
+    kv_row = wl.Hkv * wl.D * 2                      # one slot of K (or V), bf16
+    prefix = int(wl.prefix_len.sum())
+    nodes = wl.T
+    w_bytes = wl.V * wl.d * 2
+    attn_bytes = 2 * kv_row * (prefix + nodes) + 2 * nodes * wl.Hq * wl.D * 2
+    from tree_verification_jsv_b200 import synth
+    vis = 0
+    for b in range(wl.B):
+        sl = wl.request_nodes(b)
+        vis += int((wl.prefix_len[b] + synth.depths(wl.parent[sl]) + 1).sum())
+    attn_flops = 4 * wl.Hq * wl.D * vis
+    lm_bytes = w_bytes + nodes * wl.d * 2 + nodes * 8
+    lm_flops = 2 * nodes * wl.d * wl.V
+    return {
+        "north_star_bytes": 2 * kv_row * prefix + w_bytes,
+        "attention": {"bytes": attn_bytes, "flops": attn_flops},
+        "lmhead": {"bytes": lm_bytes, "flops": lm_flops},
+        "step_flops": attn_flops + lm_flops,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            ident = str(device_index)
+        self.cmd = ["nvidia-smi", "-i", ident, f"--query-gpu={','.join(CLOCK_FIELDS)}",
+                    "--format=csv,noheader,nounits", "-lms", "100"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s in self.samples:
+            if len(s) < len(CLOCK_FIELDS):
+                continue
+            try:
+                sm.append(float(s[0]))
+                mx.append(float(s[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, s[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def source_sha(*files):
+    h = hashlib.sha256()
+    for f in files:
+        h.update((ROOT / f).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key, workload, launches_units):
+    """DRAM bytes per launch from the committed ncu summary, if its source
+    hash still matches the kernel source (else None)."""
+    p = ROOT / "profiles" / "ncu_traffic.json"
+    if not p.exists():
+        return None
+    d = json.loads(p.read_text()).get(kernel_key)
+    if not d:
+        return None
+    if d.get("source_sha") != source_sha(*d["sources"]):
+        return None
+    per_unit = d["dram_bytes_per_launch"] / d["units_per_launch"]
+    return int(round(per_unit * launches_units))
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline leg)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_step(wl, tokens, g, sample_nodes):
+    """The oracle's version of one step on a bounded sample: attention of
+    every head of the first ``sample_nodes`` nodes of request 0, their LM-head
+    argmax, and the walk + compaction of request 0.  Returns nodes done."""
+    import oracle
+    n0 = int(wl.node_offsets[1])
+    ns = min(sample_nodes, n0)
+    tt, hh = np.meshgrid(np.arange(ns), np.arange(wl.Hq), indexing="ij")
+    rows = np.stack([tt.ravel(), hh.ravel()], axis=1)
+    oracle.tree_attention_wl(wl, rows=rows)
+    oracle.lmhead_top2(wl.hidden, wl.w, rows=np.arange(ns))
+    arg = np.asarray(g["argmax"], dtype=np.int64)
+    path, a, bonus = oracle.accept_path(wl.parent[:n0], tokens[:n0], arg[:n0])
+    k = wl.k_cache.copy()
+    v = wl.v_cache.copy()
+    oracle.kv_compact(k, v, wl.page_table[:1], wl.prefix_len[:1], [path])
+    return ns
+
+
+def cpu_baseline(wl, tokens, g, steps=1, sample_nodes=64):
+    import oracle
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(steps):
+        done += oracle_sample_step(wl, tokens, g, sample_nodes)
+    dt = time.perf_counter() - t0
+    ns = min(sample_nodes, int(wl.node_offsets[1]))
+    return {"value": done / dt, "unit": "nodes/s", "cores": oracle.host_threads(),
+            "kind": "oracle",
+            "sample": f"{ns} nodes of request 0 (all {wl.Hq} heads' attention + LM-head argmax over "
+                      f"{wl.V} tokens, fp64) + walk and KV compaction of request 0, x{steps}",
+            "seconds": dt}
+
+
+def run_reference(args, rank):
+    """--impl reference: the oracle as it stands, on the host cores."""
+    if rank != 0:
+        return
+    wl, tokens, g = load_workload(args.workload)
+    sample = 16
+    for _ in range(args.warmup):
+        oracle_sample_step(wl, tokens, g, sample)
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(args.steps):
+        done += oracle_sample_step(wl, tokens, g, sample)
+    dt = time.perf_counter() - t0
+    import oracle
+    value = done / dt
+    ns = min(sample, int(wl.node_offsets[1]))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "nodes/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": DESCRIPTION[args.workload], "name": args.workload,
+                   "sample_nodes_per_step": ns, "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": "nodes/s", "cores": oracle.host_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: {ns} nodes of request 0 (attention all heads + LM-head "
+                                   f"argmax, fp64) + walk and compaction of request 0"},
+        "e2e": {"value": value, "unit": "nodes/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    from tree_verification_jsv_b200 import jsv
+    from tree_verification_jsv_b200.step import VerifyStep
+
+    torch.cuda.set_device(local_rank)
+    jsv.load()
+    wl, tokens, g = load_workload(args.workload)
+    st = VerifyStep(wl, tokens, device=f"cuda:{local_rank}")
+    model = workload_model(wl)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=f"cuda:{local_rank}")
+    stream = torch.cuda.current_stream()
+
+    # correctness of this very launch configuration against stored oracle values
+    st.run()
+    torch.cuda.synchronize()
+    assert int(st.status.item()) == 0, "device-side input error"
+    assert st.argmax.cpu().numpy().tolist() == g["argmax"], "argmax differs from the oracle golden"
+    assert st.accept_len.cpu().numpy().tolist() == g["accept_len"], "accept_len differs from the oracle"
+    assert st.bonus.cpu().numpy().tolist() == g["bonus"], "bonus differs from the oracle"
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        st.run()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches0 = jsv.jsv_kernel_launches()
+    with ClockSampler(local_rank) as clocks:
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            e = ev[i]
+            e[0].record(stream)
+            st.attention()
+            e[1].record(stream)
+            st.lmhead()
+            e[2].record(stream)
+            st.accept()
+            e[3].record(stream)
+            st.compact()
+            e[4].record(stream)
+        torch.cuda.synchronize()
+    launches = jsv.jsv_kernel_launches() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    per = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)] for i in range(K)])
+    step_ms = float(per.sum(axis=1).mean())
+    call_ms = per.mean(axis=0)
+    assert int(st.status.item()) == 0
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h2d, d2h = st.h2d_bytes(), st.d2h_bytes()
+        for _ in range(3):
+            st.run_host()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            st.run_host()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        e2e = {"value_local": wl.T / (e2e_ms * 1e-3), "ms": e2e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # max over ranks
+    vals = torch.tensor([step_ms, e2e["ms"] if e2e else 0.0], dtype=torch.float64, device=f"cuda:{local_rank}")
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    step_ms_max, e2e_ms_max = float(vals[0]), float(vals[1])
+    if rank != 0:
+        return
+
+    hbm, tf_burst, tf_sus, peak_kind = peaks()
+    names = ["attention", "lmhead", "accept", "compact"]
+    share = {n: float(call_ms[j] / call_ms.sum()) for j, n in enumerate(names)}
+    dom = "lmhead" if call_ms[1] >= call_ms[0] else "attention"
+    dom_ms = float(call_ms[names.index(dom)])
+    m = model[dom]
+    t_hbm = m["bytes"] / (hbm * 1e9)
+    t_tc = m["flops"] / (tf_burst * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": m["bytes"] / (dom_ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": m["flops"] / (dom_ms * 1e-3) / 1e12, "peak": tf_burst,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = {"lmhead": "jsv_lmhead_argmax", "attention": "jsv_tree_attention"}[dom]
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
+    roof["algorithmic_bytes_per_launch"] = m["bytes"]
+    roof["algorithmic_flops_per_launch"] = m["flops"]
+    roof["traffic"] = ncu_traffic(dom, args.workload, m["bytes"])
+
+    value = world * wl.T / (step_ms_max * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "nodes/s", "n_gpus": world, "steps": K,
+        "warmup": max(args.warmup, 3), "ms_per_step": step_ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": DESCRIPTION[args.workload], "name": args.workload,
+                   "nodes_per_step": wl.T, "requests": wl.B,
+                   "prefix_tokens": int(wl.prefix_len.sum()),
+                   "l2": "flushed before every timed step (512 MB write)",
+                   "parallelism": f"replicas x{world}"},
+        "step_latency_us": step_ms_max * 1e3,
+        "step_hbm_gbs": model["north_star_bytes"] / (step_ms_max * 1e-3) / 1e9,
+        "step_hbm_frac": model["north_star_bytes"] / (step_ms_max * 1e-3) / 1e9 / hbm,
+        "step_tensor_frac": model["step_flops"] / (step_ms_max * 1e-3) / 1e12 / tf_burst,
+        "north_star_bytes": model["north_star_bytes"],
+        "call_us": {n: float(call_ms[j] * 1e3) for j, n in enumerate(names)},
+        "call_share": share,
+        "roofline": roof,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+        "accept_len": g["accept_len"][:16],
+    }
+    if e2e:
+        line["e2e"] = {"value": world * wl.T / (e2e_ms_max * 1e-3), "unit": "nodes/s",
+                       "ms_per_step": e2e_ms_max,
+                       "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                       "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, tokens, g)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

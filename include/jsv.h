@@ -1,0 +1,192 @@
+/*
+ * jsv.h -- C ABI of libjsv.so: the one-forward tree verification step of
+ * causal parallel tree drafting (JetSpec), as hand-written CUDA for sm_100a.
+ *
+ * The method (JetSpec README, "JetSpec / Overview"): a draft head proposes a
+ * token tree; the frozen target verifies the whole tree in ONE forward pass
+ * under a tree-causal attention mask, and the accepted path is chosen by the
+ * target's own logits, so decoding stays lossless.  The serving engine keeps
+ * the KV cache in pages (README, "JetSpec / Quick Start": paged KV, custom
+ * tree attention, CUDA graphs).  All reported runs are greedy (temperature 0).
+ * One verify step is four calls on one stream, in this order:
+ *
+ *   jsv_tree_attention  tree-causal attention of every node over its
+ *                       request's paged KV prefix plus its own ancestors
+ *   jsv_lmhead_argmax   LM-head projection of every node's hidden state
+ *                       fused with top-1 argmax (logits are never stored)
+ *   jsv_accept_path     greedy longest-accepted-path walk
+ *   jsv_kv_compact      move the accepted path's K/V rows to contiguous
+ *                       slots P..P+a of each request (ragged batches)
+ *
+ * Conventions for every call
+ *   - Pointers marked "device" are CUDA device (or managed) memory; the
+ *     caller allocates and owns every buffer, workspace included.  The
+ *     library never allocates, frees or synchronises.
+ *   - bf16 tensors are IEEE bfloat16 bit patterns, row-major, contiguous.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous: the return value covers host-side argument checks
+ *     and the launch only.
+ *   - Host-side checks return JSV_ERR_INVALID_ARG (NULL pointer, negative or
+ *     inconsistent size, too-small workspace) or JSV_ERR_UNSUPPORTED (a
+ *     shape outside the supported set) and launch nothing.
+ *   - Errors that only the device can see (a malformed parent array, a page
+ *     index outside [0, num_pages), node offsets that disagree with
+ *     total_nodes, a path longer than max_path) are written to
+ *     batch->dev_status (if non-NULL) with an atomic compare-and-swap from
+ *     0, so the first error sticks; the affected request's work is skipped.
+ *     Kernels never trap.  The caller zeroes *dev_status before a step.
+ *   - Calls on distinct streams with distinct workspaces and outputs may run
+ *     concurrently.
+ */
+#ifndef JSV_H
+#define JSV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define JSV_API __attribute__((visibility("default")))
+#else
+#define JSV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    JSV_OK = 0,
+    JSV_ERR_INVALID_ARG = 1,   /* host-visible bad argument                  */
+    JSV_ERR_UNSUPPORTED = 2,   /* shape outside the supported set            */
+    JSV_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed       */
+    JSV_ERR_TIMEOUT = 4,       /* a bounded device wait gave up              */
+    JSV_ERR_DEVICE_INPUT = 5   /* written to *dev_status: bad device data    */
+} jsv_status;
+
+/*
+ * Geometry of one verify step over B requests, shared by the calls that
+ * touch the tree or the cache.
+ *
+ * Notation: request b has P_b committed prefix tokens and a draft tree of
+ * N_b nodes (node 0 = root = the last committed token, whose K/V this
+ * forward computes).  Nodes of all requests are packed: request b owns
+ * global nodes node_offsets[b] .. node_offsets[b+1]-1, T = node_offsets[B].
+ *
+ * Tree: parent[] holds request-local indices with parent[0] = -1 and
+ * 0 <= parent[i] < i for i > 0 (any topological order).
+ *
+ * Cache: k_cache and v_cache are [num_pages][page_size][Hkv][D] bf16.
+ * Logical slot s of request b is row s % page_size of physical page
+ * page_table[b * max_pages_per_req + s / page_size].  Slots [0, P_b) hold
+ * the prefix; the caller has written tree node j's K/V at slot P_b + j, so
+ * pages covering [0, P_b + N_b) must be mapped.
+ */
+typedef struct {
+    int32_t B;                   /* requests, >= 1                                */
+    int32_t Hq, Hkv, D;          /* query heads, KV heads (Hq % Hkv == 0), D in {64,128} */
+    int32_t page_size;           /* must be 16                                    */
+    int32_t max_pages_per_req;   /* row stride of page_table                      */
+    int32_t num_pages;           /* physical pages in k_cache and in v_cache      */
+    int32_t total_nodes;         /* T, must equal node_offsets[B]                 */
+    int32_t max_nodes;           /* upper bound on N_b, 1..512                    */
+    int32_t max_prefix;          /* upper bound on P_b, >= 0                      */
+    const int32_t *page_table;   /* device [B][max_pages_per_req]                 */
+    const int32_t *prefix_len;   /* device [B]   P_b                              */
+    const int32_t *node_offsets; /* device [B+1]                                  */
+    const int32_t *parent;       /* device [T]   request-local parent index       */
+    int32_t *dev_status;         /* device [1] or NULL: first device-side error   */
+} jsv_batch;
+
+/* Bytes of scratch jsv_tree_attention needs for this geometry (split-KV
+ * partial results).  Depends only on the host-side fields. */
+JSV_API size_t jsv_tree_attention_workspace_size(const jsv_batch *batch);
+
+/*
+ * Tree-causal attention (README, "JetSpec / Overview": one forward pass under
+ * a tree-causal mask).  For request b, node i, query head h, with
+ * g = h / (Hq / Hkv), the visible sequence is prefix slots 0..P_b-1 followed
+ * by slots P_b + j for every j on the root..i path (i included):
+ *     out[t][h] = sum_j softmax_j(scale * <q[t][h], k_j>) * v_j
+ * computed in fp32 from bf16 inputs and rounded to bf16.
+ *   q        device [T][Hq][D] bf16, post-rotary
+ *   k_cache, v_cache  device caches as described above (read only)
+ *   scale    softmax scale (normally 1/sqrt(D))
+ *   out      device [T][Hq][D] bf16
+ *   workspace, workspace_bytes  device scratch of at least
+ *            jsv_tree_attention_workspace_size(batch) bytes, 256-B aligned
+ */
+JSV_API jsv_status jsv_tree_attention(const jsv_batch *batch, const uint16_t *q,
+                              const uint16_t *k_cache, const uint16_t *v_cache,
+                              float scale, uint16_t *out,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of scratch jsv_lmhead_argmax needs (one 64-bit key per node). */
+JSV_API size_t jsv_lmhead_argmax_workspace_size(int32_t T, int32_t d, int32_t V);
+
+/*
+ * LM head fused with top-1 argmax (README, "JetSpec / Overview": the path is
+ * selected by the target's own logits; temperature 0).
+ *     argmax[t] = smallest v attaining max_v sum_k hidden[t][k] * w[v][k]
+ * accumulated in fp32 from bf16; logits are never written to memory.
+ *   hidden     device [T][d] bf16
+ *   w          device [V][d] bf16 (the LM-head weight, row per token)
+ *   argmax     device [T] int32
+ *   max_logit  device [T] float (the fp32 maximum) or NULL
+ *   workspace  device scratch of jsv_lmhead_argmax_workspace_size() bytes,
+ *              8-B aligned; the call initialises it
+ * Supported: 1 <= T, d % 64 == 0, 64 <= d <= 16384, 1 <= V < 2^31.
+ */
+JSV_API jsv_status jsv_lmhead_argmax(const uint16_t *hidden, const uint16_t *w,
+                             int32_t T, int32_t d, int32_t V,
+                             int32_t *argmax, float *max_logit,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Greedy accept walk (README, "JetSpec / Overview": lossless by
+ * construction; "tokens per forward" = accepted + 1).  Per request, start at
+ * the root (always accepted); while some child c of the current node has
+ * tokens[c] == argmax[current], move to the smallest such c.
+ *   tokens      device [T] int32, the draft token of every node
+ *   argmax      device [T] int32, the target's choice at every node
+ *   max_path    row length of `path` (>= 1)
+ *   path        device [B][max_path] int32: request-local indices of the
+ *               accepted path starting with 0, then -1 padding
+ *   accept_len  device [B] int32: accepted draft nodes a = path length - 1
+ *   bonus       device [B] int32: argmax at the last accepted node
+ * A path that would exceed max_path sets JSV_ERR_DEVICE_INPUT and is cut.
+ */
+JSV_API jsv_status jsv_accept_path(const jsv_batch *batch, const int32_t *tokens,
+                           const int32_t *argmax, int32_t max_path,
+                           int32_t *path, int32_t *accept_len, int32_t *bonus,
+                           void *stream);
+
+/*
+ * Accepted-path KV compaction (README, "JetSpec / Quick Start": paged KV).
+ * For every request and k = 0..a: the K and V rows (all KV heads) of slot
+ * P_b + path[k] move to slot P_b + k, with the result of an in-order copy
+ * (every source is read before any destination is written).  Slots other
+ * than P_b..P_b+a are untouched.  new_len[b] = P_b + a + 1.
+ *   k_cache, v_cache  device caches, updated in place
+ *   path, accept_len  as written by jsv_accept_path (max_path = row stride)
+ *   new_len           device [B] int32
+ */
+JSV_API jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uint16_t *v_cache,
+                          const int32_t *path, int32_t max_path, const int32_t *accept_len,
+                          int32_t *new_len, void *stream);
+
+/* Number of kernels this library has launched in the calling process since
+ * it was loaded (all devices, all streams).  A diagnostic for counting the
+ * launches inside a timed region; not tied to any stream order. */
+JSV_API uint64_t jsv_kernel_launches(void);
+
+/* Static string for a status code. */
+JSV_API const char *jsv_status_string(jsv_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+JSV_API int32_t jsv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JSV_H */

@@ -1,0 +1,201 @@
+"""GPU edge cases through the C ABI: tiny and degenerate trees, ragged
+prefixes that are not multiples of the page size, trees crossing page
+boundaries, sharp attention, head-dim 64, G = 1, vocabulary and node counts
+that are not tile multiples, and device-side error reporting."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import attention_close, bf16, small_case
+from tree_verification_jsv_b200 import jsv, synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from tree_verification_jsv_b200 import build
+    build.build()
+    jsv.load()
+
+
+def _dev_i32(x):
+    return torch.as_tensor(np.ascontiguousarray(x, dtype=np.int32)).cuda()
+
+
+def _dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits, dtype=np.uint16).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _bits(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _batch(case, status, **over):
+    offs = case["node_offsets"]
+    n = np.diff(offs)
+    dev = dict(page_table=_dev_i32(case["page_table"]), prefix_len=_dev_i32(case["prefix_len"]),
+               node_offsets=_dev_i32(offs), parent=_dev_i32(case["parent"]))
+    kw = dict(B=len(n), Hq=case["Hq"], Hkv=case["Hkv"], D=case["D"],
+              max_pages_per_req=case["page_table"].shape[1], num_pages=case["num_pages"],
+              total_nodes=int(offs[-1]), max_nodes=int(n.max()),
+              max_prefix=int(max(case["prefix_len"])), dev_status=status, **dev)
+    kw.update(over)
+    return jsv.make_batch(**kw), dev
+
+
+def run_attention(case, **over):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    batch, keep = _batch(case, status, **over)
+    q = _dev_bf16(case["q"])
+    k = _dev_bf16(case["k_cache"])
+    v = _dev_bf16(case["v_cache"])
+    T = int(case["node_offsets"][-1])
+    out = torch.zeros((T, case["Hq"], case["D"]), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(256, jsv.jsv_tree_attention_workspace_size(batch)), dtype=torch.uint8, device="cuda")
+    jsv.jsv_tree_attention(batch, q, k, v, case["scale"], out, ws)
+    torch.cuda.synchronize()
+    return synth.bf16_bits_to_f32(_bits(out)).astype(np.float64), int(status.item())
+
+
+ATTN_CASES = {
+    "single_node_no_prefix": ([np.array([-1])], [0], 4, 2, 128),
+    "root_only_prefix_17": ([np.array([-1])], [17], 4, 2, 128),
+    "chain_cross_pages": ([np.arange(-1, 40)], [29], 8, 2, 128),
+    "ragged_three": ([synth.tiny_tree(np.random.default_rng(1), 23, 6, 3),
+                      np.array([-1, 0]), synth.tiny_tree(np.random.default_rng(2), 70, 9, 4)],
+                     [1, 0, 300], 8, 2, 128),
+    "head_dim_64_g1": ([synth.tiny_tree(np.random.default_rng(3), 31, 5, 3)], [45], 4, 4, 64),
+    "g8_long": ([synth.budget_tree(np.random.default_rng(4), 100, 10, 4)], [1500], 16, 2, 128),
+    "max_nodes_512": ([synth.budget_tree(np.random.default_rng(5), 512, 16, 8)], [64], 2, 1, 64),
+}
+
+
+@pytest.mark.parametrize("name", list(ATTN_CASES))
+@pytest.mark.parametrize("sharp", [False, True])
+def test_attention_edge_cases(name, sharp):
+    parents, pre, Hq, Hkv, D = ATTN_CASES[name]
+    case = small_case(parents, pre, Hq=Hq, Hkv=Hkv, D=D, seed=11,
+                      q_scale=4.0 * math.sqrt(D) if sharp else 1.0)
+    got, st = run_attention(case)
+    assert st == 0
+    from helpers import run_oracle_attention
+    attention_close(got, run_oracle_attention(case), name)
+
+
+@pytest.mark.parametrize("T,d,V", [(1, 64, 1), (5, 128, 1000), (16, 256, 1024), (64, 512, 4099),
+                                   (130, 192, 3000), (300, 1024, 20000)])
+def test_lmhead_argmax_shapes(T, d, V):
+    rng = np.random.default_rng(T * 7 + V)
+    H = bf16(rng.standard_normal((T, d)) / math.sqrt(d))
+    W = bf16(rng.standard_normal((V, d)) / math.sqrt(d))
+    a, t1, t2 = oracle.lmhead_top2(H, W)
+    ok, _ = oracle.certify_margin(H, W, a, t1, t2)
+    assert ok.mean() > 0.8
+    arg = torch.empty(T, dtype=torch.int32, device="cuda")
+    ml = torch.empty(T, dtype=torch.float32, device="cuda")
+    ws = torch.empty(jsv.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
+    jsv.jsv_lmhead_argmax(_dev_bf16(H), _dev_bf16(W), T, d, V, arg, ml, ws)
+    torch.cuda.synchronize()
+    g = arg.cpu().numpy()
+    assert np.array_equal(g[ok], a[ok])
+    assert np.all((g >= 0) & (g < V))
+    assert np.allclose(ml.cpu().numpy()[ok], t1[ok], rtol=1e-4, atol=1e-5)
+
+
+def test_lmhead_ties_take_smallest_index():
+    d, V, T = 64, 700, 3
+    W = np.zeros((V, d), dtype=np.float32)
+    W[[17, 300, 650]] = 1.0 / 8          # exact ties for every node
+    H = np.full((T, d), 1.0 / 8, dtype=np.float32)
+    arg = torch.empty(T, dtype=torch.int32, device="cuda")
+    ws = torch.empty(jsv.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
+    jsv.jsv_lmhead_argmax(_dev_bf16(bf16(H)), _dev_bf16(bf16(W)), T, d, V, arg, None, ws)
+    torch.cuda.synchronize()
+    assert arg.cpu().tolist() == [17, 17, 17]
+
+
+def _walk_and_compact(parents, pre, tokens, argmax, max_path=None):
+    case = small_case(parents, pre, Hq=2, Hkv=2, D=64, seed=3)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    batch, keep = _batch(case, status)
+    B = len(parents)
+    mp = max_path or max(len(p) for p in parents)
+    path = torch.full((B, mp), 77, dtype=torch.int32, device="cuda")
+    acc = torch.empty(B, dtype=torch.int32, device="cuda")
+    bonus = torch.empty(B, dtype=torch.int32, device="cuda")
+    nl = torch.empty(B, dtype=torch.int32, device="cuda")
+    k, v = _dev_bf16(case["k_cache"]), _dev_bf16(case["v_cache"])
+    jsv.jsv_accept_path(batch, _dev_i32(tokens), _dev_i32(argmax), mp, path, acc, bonus)
+    jsv.jsv_kv_compact(batch, k, v, path, mp, acc, nl)
+    torch.cuda.synchronize()
+    return case, dict(path=path.cpu().numpy(), acc=acc.cpu().numpy(), bonus=bonus.cpu().numpy(),
+                      new_len=nl.cpu().numpy(), k=_bits(k), v=_bits(v), status=int(status.item()))
+
+
+def test_walk_and_compaction_random_batches():
+    rng = np.random.default_rng(9)
+    for trial in range(6):
+        B = int(rng.integers(1, 9))
+        parents = [synth.tiny_tree(rng, int(rng.integers(1, 200)), 40, 3) for _ in range(B)]
+        pre = [int(rng.integers(0, 100)) for _ in range(B)]
+        T = sum(len(p) for p in parents)
+        argmax = rng.integers(0, 6, T)        # small vocab: duplicates and long paths
+        tokens = rng.integers(0, 6, T)
+        offs = np.concatenate([[0], np.cumsum([len(p) for p in parents])])
+        for b, p in enumerate(parents):
+            for c in range(1, len(p)):
+                if rng.random() < 0.8:
+                    tokens[offs[b] + c] = argmax[offs[b] + p[c]]
+        case, got = _walk_and_compact(parents, pre, tokens, argmax)
+        assert got["status"] == 0
+        ref = oracle.accept_batch(offs, np.concatenate(parents), tokens, argmax)
+        kref, vref = case["k_cache"].copy(), case["v_cache"].copy()
+        nl = oracle.kv_compact(kref, vref, case["page_table"], case["prefix_len"], [r[0] for r in ref])
+        for b, (p, a, bo) in enumerate(ref):
+            assert got["acc"][b] == a and got["bonus"][b] == bo
+            assert got["path"][b, :a + 1].tolist() == p
+        assert np.array_equal(got["new_len"], nl)
+        assert np.array_equal(got["k"], kref) and np.array_equal(got["v"], vref)
+
+
+def test_full_depth_chain_and_zero_accept():
+    n = 300
+    chain = np.arange(-1, n - 1)
+    argmax = np.arange(n) + 1000
+    tokens = np.concatenate([[5], argmax[:-1]])                 # everything matches
+    case, got = _walk_and_compact([chain, np.array([-1, 0, 0])], [33, 7],
+                                  np.concatenate([tokens, [1, 2, 3]]),
+                                  np.concatenate([argmax, [9, 9, 9]]))
+    assert got["status"] == 0
+    assert got["acc"].tolist() == [n - 1, 0]
+    assert got["path"][0].tolist() == list(range(n))
+    assert got["new_len"].tolist() == [33 + n, 8]
+
+
+def test_path_longer_than_max_path_is_reported():
+    n = 10
+    chain = np.arange(-1, n - 1)
+    argmax = np.arange(n) + 50
+    tokens = np.concatenate([[0], argmax[:-1]])
+    case, got = _walk_and_compact([chain], [3], tokens, argmax, max_path=4)
+    assert got["status"] == jsv.JSV_ERR_DEVICE_INPUT
+    assert got["path"][0].tolist() == [0, 1, 2, 3]
+
+
+def test_malformed_parent_is_reported_not_trapped():
+    case = small_case([np.array([-1, 0, 1, 1])], [20], Hq=2, Hkv=1, D=64, seed=4)
+    case["parent"] = np.array([-1, 0, 3, 1], dtype=np.int32)    # parent[2] = 3 > 2
+    out, st = run_attention(case)
+    assert st == jsv.JSV_ERR_DEVICE_INPUT
+
+
+def test_page_out_of_range_is_reported():
+    case = small_case([np.array([-1, 0])], [40], Hq=2, Hkv=1, D=64, seed=5)
+    case["page_table"] = case["page_table"].copy()
+    case["page_table"][0, 1] = case["num_pages"] + 5
+    out, st = run_attention(case)
+    assert st == jsv.JSV_ERR_DEVICE_INPUT

@@ -1,0 +1,80 @@
+// Greedy accept walk: one warp per request.
+//
+// JetSpec README, "JetSpec / Overview": the accepted path is chosen by the
+// target's own logits, so decoding is lossless.  At temperature 0 that is
+// the greedy descent: from the root, step to the smallest-index child whose
+// draft token equals the target's argmax at the current node, until no
+// child matches.  Children have larger indices than their parent
+// (topological order), so each step scans indices > cur with a warp ballot
+// and takes the lowest set lane of the first chunk that has a match.
+#include "jsv_internal.cuh"
+
+namespace jsv {
+
+__global__ void __launch_bounds__(128)
+accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
+                   const int32_t *__restrict__ argmax, int max_path, int32_t *__restrict__ path,
+                   int32_t *__restrict__ accept_len, int32_t *__restrict__ bonus) {
+    const int warps = blockDim.x >> 5;
+    const int b = blockIdx.x * warps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (b >= a.B) return;
+    int32_t *row = path + (size_t)b * max_path;
+
+    Request r;
+    bool ok = load_request(a, b, r);
+    if (ok) {
+        bool bad = false;
+        for (int j = lane; j < r.n; j += 32) {
+            int p = a.parent[r.base + j];
+            bad |= (j == 0) ? (p != -1) : (p < 0 || p >= j);
+        }
+        if (__any_sync(0xffffffffu, bad)) {
+            if (lane == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+            ok = false;
+        }
+    }
+    if (!ok) {
+        for (int k = lane; k < max_path; k += 32) row[k] = k == 0 ? 0 : -1;
+        if (lane == 0) { accept_len[b] = 0; bonus[b] = -1; }
+        return;
+    }
+
+    int cur = 0, len = 1;
+    while (true) {
+        const int want = argmax[r.base + cur];
+        int found = -1;
+        for (int j0 = cur + 1; j0 < r.n; j0 += 32) {
+            const int j = j0 + lane;
+            const bool m = j < r.n && a.parent[r.base + j] == cur && tokens[r.base + j] == want;
+            const unsigned bal = __ballot_sync(0xffffffffu, m);
+            if (bal) { found = j0 + __ffs(bal) - 1; break; }
+        }
+        if (found < 0) break;
+        if (len >= max_path) {
+            if (lane == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+            break;
+        }
+        if (lane == 0) row[len] = found;
+        ++len;
+        cur = found;
+    }
+    if (lane == 0) {
+        row[0] = 0;
+        accept_len[b] = len - 1;
+        bonus[b] = argmax[r.base + cur];
+    }
+    for (int k = len + lane; k < max_path; k += 32) row[k] = -1;
+}
+
+cudaError_t launch_accept_path(const BatchArgs &a, const int32_t *tokens, const int32_t *argmax,
+                               int max_path, int32_t *path, int32_t *accept_len, int32_t *bonus,
+                               cudaStream_t st) {
+    const int warps = 4;
+    dim3 grid((a.B + warps - 1) / warps);
+    accept_path_kernel<<<grid, warps * 32, 0, st>>>(a, tokens, argmax, max_path, path, accept_len, bonus);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace jsv

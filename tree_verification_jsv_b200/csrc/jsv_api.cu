@@ -1,0 +1,113 @@
+// C ABI of libjsv.so: host-side argument checks, then one launch sequence
+// per call on the caller's stream.  See include/jsv.h for the contract.
+#include "jsv_internal.cuh"
+
+#include <atomic>
+
+namespace jsv {
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace jsv
+
+namespace {
+
+bool aligned(const void *p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+jsv_status check_batch(const jsv_batch *b) {
+    if (!b) return JSV_ERR_INVALID_ARG;
+    if (b->B < 1 || b->Hq < 1 || b->Hkv < 1 || b->total_nodes < b->B || b->max_nodes < 1 ||
+        b->max_prefix < 0 || b->max_pages_per_req < 1 || b->num_pages < 1)
+        return JSV_ERR_INVALID_ARG;
+    if (b->Hq % b->Hkv != 0) return JSV_ERR_INVALID_ARG;
+    if (b->D != 64 && b->D != 128) return JSV_ERR_UNSUPPORTED;
+    if (b->page_size != 16) return JSV_ERR_UNSUPPORTED;
+    if (b->max_nodes > 512) return JSV_ERR_UNSUPPORTED;
+    if ((long long)b->max_pages_per_req * b->page_size < 1) return JSV_ERR_INVALID_ARG;
+    if (!b->page_table || !b->prefix_len || !b->node_offsets || !b->parent) return JSV_ERR_INVALID_ARG;
+    return JSV_OK;
+}
+
+jsv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? JSV_OK : JSV_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t jsv_tree_attention_workspace_size(const jsv_batch *batch) {
+    if (check_batch(batch) != JSV_OK) return 0;
+    return jsv::attention_workspace_bytes(jsv::to_args(batch));
+}
+
+jsv_status jsv_tree_attention(const jsv_batch *batch, const uint16_t *q, const uint16_t *k_cache,
+                              const uint16_t *v_cache, float scale, uint16_t *out, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+    jsv_status s = check_batch(batch);
+    if (s != JSV_OK) return s;
+    if (!q || !k_cache || !v_cache || !out) return JSV_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
+        return JSV_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || scale != scale) return JSV_ERR_INVALID_ARG;
+    const jsv::BatchArgs a = jsv::to_args(batch);
+    const size_t need = jsv::attention_workspace_bytes(a);
+    if (workspace_bytes < need || (need && (!workspace || !aligned(workspace, 256))))
+        return JSV_ERR_INVALID_ARG;
+    return from_cuda(jsv::launch_tree_attention(a, q, k_cache, v_cache, scale, out, workspace,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+size_t jsv_lmhead_argmax_workspace_size(int32_t T, int32_t d, int32_t V) {
+    if (T < 1 || d < 1 || V < 1) return 0;
+    return jsv::lmhead_workspace_bytes(T, d, V);
+}
+
+jsv_status jsv_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int32_t T, int32_t d,
+                             int32_t V, int32_t *argmax, float *max_logit, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    if (!hidden || !w || !argmax || T < 1 || d < 1 || V < 1) return JSV_ERR_INVALID_ARG;
+    if (d % 64 != 0 || d > 16384) return JSV_ERR_UNSUPPORTED;
+    if (!aligned(hidden, 16) || !aligned(w, 16)) return JSV_ERR_INVALID_ARG;
+    const size_t need = jsv::lmhead_workspace_bytes(T, d, V);
+    if (workspace_bytes < need || !workspace || !aligned(workspace, 8)) return JSV_ERR_INVALID_ARG;
+    return from_cuda(jsv::launch_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, workspace,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+jsv_status jsv_accept_path(const jsv_batch *batch, const int32_t *tokens, const int32_t *argmax,
+                           int32_t max_path, int32_t *path, int32_t *accept_len, int32_t *bonus,
+                           void *stream) {
+    jsv_status s = check_batch(batch);
+    if (s != JSV_OK) return s;
+    if (!tokens || !argmax || !path || !accept_len || !bonus || max_path < 1) return JSV_ERR_INVALID_ARG;
+    return from_cuda(jsv::launch_accept_path(jsv::to_args(batch), tokens, argmax, max_path, path,
+                                             accept_len, bonus, static_cast<cudaStream_t>(stream)));
+}
+
+jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uint16_t *v_cache,
+                          const int32_t *path, int32_t max_path, const int32_t *accept_len,
+                          int32_t *new_len, void *stream) {
+    jsv_status s = check_batch(batch);
+    if (s != JSV_OK) return s;
+    if (!k_cache || !v_cache || !path || !accept_len || !new_len || max_path < 1)
+        return JSV_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return JSV_ERR_INVALID_ARG;
+    return from_cuda(jsv::launch_kv_compact(jsv::to_args(batch), k_cache, v_cache, path, max_path,
+                                            accept_len, new_len, static_cast<cudaStream_t>(stream)));
+}
+
+const char *jsv_status_string(jsv_status status) {
+    switch (status) {
+        case JSV_OK: return "ok";
+        case JSV_ERR_INVALID_ARG: return "invalid argument";
+        case JSV_ERR_UNSUPPORTED: return "unsupported shape";
+        case JSV_ERR_CUDA: return "CUDA error";
+        case JSV_ERR_TIMEOUT: return "device wait timed out";
+        case JSV_ERR_DEVICE_INPUT: return "malformed device-side input";
+    }
+    return "unknown status";
+}
+
+int32_t jsv_version(void) { return 100; }
+
+uint64_t jsv_kernel_launches(void) { return jsv::g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

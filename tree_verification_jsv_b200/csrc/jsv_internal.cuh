@@ -1,0 +1,90 @@
+// Internal helpers shared by the libjsv.so kernels (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/jsv.h"
+
+namespace jsv {
+
+// Device-side copy of the host-visible batch geometry (passed by value).
+struct BatchArgs {
+    int B, Hq, Hkv, D, page_size, max_pages_per_req, num_pages, total_nodes, max_nodes, max_prefix;
+    const int32_t *page_table, *prefix_len, *node_offsets, *parent;
+    int32_t *dev_status;
+};
+
+inline BatchArgs to_args(const jsv_batch *b) {
+    BatchArgs a;
+    a.B = b->B; a.Hq = b->Hq; a.Hkv = b->Hkv; a.D = b->D; a.page_size = b->page_size;
+    a.max_pages_per_req = b->max_pages_per_req; a.num_pages = b->num_pages;
+    a.total_nodes = b->total_nodes; a.max_nodes = b->max_nodes; a.max_prefix = b->max_prefix;
+    a.page_table = b->page_table; a.prefix_len = b->prefix_len; a.node_offsets = b->node_offsets;
+    a.parent = b->parent; a.dev_status = b->dev_status;
+    return a;
+}
+
+__device__ __forceinline__ void flag_error(int32_t *status, int code) {
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
+    return __uint_as_float(((uint32_t)h) << 16);
+}
+
+// Request geometry read from device arrays, with the checks every kernel
+// needs before touching the request's memory.  Returns false (and flags the
+// status word) if the request's descriptors are inconsistent.
+struct Request {
+    int base, n, P;
+};
+
+__device__ __forceinline__ bool load_request(const BatchArgs &a, int b, Request &r) {
+    int s = a.node_offsets[b], e = a.node_offsets[b + 1];
+    int P = a.prefix_len[b];
+    bool ok = s >= 0 && e > s && e <= a.total_nodes && (e - s) <= a.max_nodes &&
+              P >= 0 && P <= a.max_prefix &&
+              (P + (e - s) + a.page_size - 1) / a.page_size <= a.max_pages_per_req;
+    if (b == a.B - 1 && e != a.total_nodes) ok = false;
+    if (!ok) {
+        flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+        return false;
+    }
+    r.base = s; r.n = e - s; r.P = P;
+    return true;
+}
+
+// Physical row index (page * page_size + offset) of logical slot s, or -1
+// (flagged) if the page entry is out of range.
+__device__ __forceinline__ long long slot_phys_row(const BatchArgs &a, int b, int s) {
+    int page = a.page_table[(size_t)b * a.max_pages_per_req + s / a.page_size];
+    if (page < 0 || page >= a.num_pages) {
+        flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+        return -1;
+    }
+    return (long long)page * a.page_size + (s % a.page_size);
+}
+
+// Count of kernel launches issued by the library (see jsv_kernel_launches).
+void count_launches(int n);
+
+}  // namespace jsv
+
+// Launchers (defined in the kernel files, called from jsv_api.cu).
+namespace jsv {
+cudaError_t launch_accept_path(const BatchArgs &a, const int32_t *tokens, const int32_t *argmax,
+                               int max_path, int32_t *path, int32_t *accept_len, int32_t *bonus,
+                               cudaStream_t st);
+cudaError_t launch_kv_compact(const BatchArgs &a, uint16_t *k_cache, uint16_t *v_cache,
+                              const int32_t *path, int max_path, const int32_t *accept_len,
+                              int32_t *new_len, cudaStream_t st);
+size_t lmhead_workspace_bytes(int T, int d, int V);
+cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int T, int d, int V,
+                                 int32_t *argmax, float *max_logit, void *ws, cudaStream_t st);
+size_t attention_workspace_bytes(const BatchArgs &a);
+cudaError_t launch_tree_attention(const BatchArgs &a, const uint16_t *q, const uint16_t *k_cache,
+                                  const uint16_t *v_cache, float scale, uint16_t *out, void *ws,
+                                  cudaStream_t st);
+}  // namespace jsv

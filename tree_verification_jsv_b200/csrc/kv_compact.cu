@@ -1,0 +1,103 @@
+// Accepted-path KV compaction, in place in the paged cache.
+//
+// Paged KV per the JetSpec README ("JetSpec / Quick Start"); the ragged
+// batch motivation (requests accept different numbers of tokens, so their
+// caches must be re-synchronised) per the EXSPEC/EQSPEC abstract.  For
+// k = 0..a the row at slot P + path[k] moves to slot P + k.  The path is
+// strictly increasing with path[0] = 0, so path[k] >= k: a source can only
+// be clobbered by the destination of an EARLIER k.  Each CTA therefore
+// moves the rows in chunks of increasing k and, inside a chunk, reads every
+// source into shared memory before writing any destination.  A later chunk
+// never reads a slot an earlier chunk wrote (its sources are >= its own k,
+// which exceeds every earlier destination).
+//
+// Grid: (request, K-or-V, KV-head group).  A row of one KV head is D bf16
+// (128 or 256 bytes) moved as 16-byte vectors.
+#include "jsv_internal.cuh"
+
+namespace jsv {
+
+constexpr int kCompactThreads = 256;
+constexpr int kCompactChunk = 64;        // rows per chunk
+constexpr int kHeadsPerCta = 2;
+
+__global__ void __launch_bounds__(kCompactThreads)
+kv_compact_kernel(BatchArgs a, uint16_t *__restrict__ k_cache, uint16_t *__restrict__ v_cache,
+                  const int32_t *__restrict__ path, int max_path,
+                  const int32_t *__restrict__ accept_len, int32_t *__restrict__ new_len) {
+    extern __shared__ uint4 stage[];      // [kCompactChunk][heads][D/8]
+    __shared__ int s_src[kCompactChunk], s_dst[kCompactChunk];
+    __shared__ int s_ok;
+    const int b = blockIdx.x;
+    uint16_t *cache = blockIdx.y == 0 ? k_cache : v_cache;
+    const int h0 = blockIdx.z * kHeadsPerCta;
+    const int heads = min(kHeadsPerCta, a.Hkv - h0);
+    const int vec_per_head = a.D / 8;
+    const int vec_per_row = heads * vec_per_head;
+
+    Request r;
+    if (threadIdx.x == 0) {
+        int ok = load_request(a, b, r) ? 1 : 0;
+        int acc = ok ? accept_len[b] : 0;
+        if (ok && (acc < 0 || acc >= r.n || acc + 1 > max_path)) {
+            flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+            ok = 0;
+        }
+        const int32_t *row = path + (size_t)b * max_path;
+        if (ok && row[0] != 0) ok = 0;
+        for (int k = 1; ok && k <= acc; ++k)
+            if (row[k] <= row[k - 1] || row[k] >= r.n) ok = 0;
+        if (!ok) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+        // every page the move touches (slots P .. P+n-1) must be mapped
+        if (ok) {
+            for (int pg = r.P / a.page_size; ok && pg <= (r.P + r.n - 1) / a.page_size; ++pg)
+                if (slot_phys_row(a, b, pg * a.page_size) < 0) ok = 0;
+        }
+        s_ok = ok;
+        if (ok && blockIdx.y == 0 && blockIdx.z == 0) new_len[b] = r.P + acc + 1;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+    load_request(a, b, r);
+    const int acc = accept_len[b];
+    const int32_t *row = path + (size_t)b * max_path;
+
+    for (int k0 = 0; k0 <= acc; k0 += kCompactChunk) {
+        const int rows = min(kCompactChunk, acc + 1 - k0);
+        for (int i = threadIdx.x; i < rows; i += blockDim.x) {
+            s_src[i] = (int)slot_phys_row(a, b, r.P + row[k0 + i]);
+            s_dst[i] = (int)slot_phys_row(a, b, r.P + k0 + i);
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < rows * vec_per_row; e += blockDim.x) {
+            const int i = e / vec_per_row, c = e % vec_per_row;
+            const int hh = c / vec_per_head, x = c % vec_per_head;
+            if (s_src[i] == s_dst[i]) continue;
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                cache + ((size_t)s_src[i] * a.Hkv + h0 + hh) * a.D);
+            stage[e] = src[x];
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < rows * vec_per_row; e += blockDim.x) {
+            const int i = e / vec_per_row, c = e % vec_per_row;
+            const int hh = c / vec_per_head, x = c % vec_per_head;
+            if (s_src[i] == s_dst[i]) continue;
+            uint4 *dst = reinterpret_cast<uint4 *>(cache + ((size_t)s_dst[i] * a.Hkv + h0 + hh) * a.D);
+            dst[x] = stage[e];
+        }
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_kv_compact(const BatchArgs &a, uint16_t *k_cache, uint16_t *v_cache,
+                              const int32_t *path, int max_path, const int32_t *accept_len,
+                              int32_t *new_len, cudaStream_t st) {
+    dim3 grid(a.B, 2, (a.Hkv + kHeadsPerCta - 1) / kHeadsPerCta);
+    size_t smem = (size_t)kCompactChunk * kHeadsPerCta * (a.D / 8) * sizeof(uint4);
+    kv_compact_kernel<<<grid, kCompactThreads, smem, st>>>(a, k_cache, v_cache, path, max_path,
+                                                            accept_len, new_len);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace jsv
