@@ -174,6 +174,33 @@ JSV_API jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uin
                           const int32_t *path, int32_t max_path, const int32_t *accept_len,
                           int32_t *new_len, void *stream);
 
+/*
+ * LM head fused with top-1 argmax for callers that cannot allocate device
+ * memory (a region under CUDA-graph capture, a plugin whose host owns every
+ * allocation, a loop that cannot afford cudaMalloc's synchronisation).
+ * The pages have no counterpart: it is a deployment variant of
+ * jsv_lmhead_argmax with the same result, whose scratch (one 64-bit key per
+ * node) is a fixed file-scope device array inside the library instead of a
+ * workspace argument.  The caller still passes inputs and outputs.
+ *   - T must be <= JSV_NOALLOC_MAX_NODES, else JSV_ERR_UNSUPPORTED; the
+ *     other arguments follow jsv_lmhead_argmax.
+ *   - The array (JSV_NOALLOC_MAX_NODES * 8 bytes) is held on every GPU that
+ *     loads the library until the process exits.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
+ *     library routine.  Each call clears the keys it uses before its kernel.
+ *   - Every call shares the one array, which keeps the last call's contents:
+ *     calls whose kernels overlap on the GPU (different streams, or
+ *     different host threads on one device) race and give wrong results.
+ *     Serialise them on one stream.
+ */
+#define JSV_NOALLOC_MAX_NODES 8192
+JSV_API jsv_status jsv_lmhead_argmax_noalloc(const uint16_t *hidden, const uint16_t *w,
+                                             int32_t T, int32_t d, int32_t V,
+                                             int32_t *argmax, float *max_logit, void *stream);
+
 /* Number of kernels this library has launched in the calling process since
  * it was loaded (all devices, all streams).  A diagnostic for counting the
  * launches inside a timed region; not tied to any stream order. */

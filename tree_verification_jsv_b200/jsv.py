@@ -22,7 +22,11 @@ JSV_ERR_DEVICE_INPUT = 5
 
 EXPORTS = ("jsv_tree_attention_workspace_size", "jsv_tree_attention",
            "jsv_lmhead_argmax_workspace_size", "jsv_lmhead_argmax", "jsv_accept_path",
-           "jsv_kv_compact", "jsv_status_string", "jsv_version", "jsv_kernel_launches")
+           "jsv_kv_compact", "jsv_status_string", "jsv_version", "jsv_kernel_launches",
+           "jsv_lmhead_argmax_noalloc")
+
+# Largest node count jsv_lmhead_argmax_noalloc accepts (JSV_NOALLOC_MAX_NODES).
+NOALLOC_MAX_NODES = 8192
 
 
 class JsvError(RuntimeError):
@@ -72,6 +76,8 @@ def load() -> ctypes.CDLL:
     lib.jsv_status_string.restype = ctypes.c_char_p
     lib.jsv_version.argtypes = []
     lib.jsv_version.restype = i32
+    lib.jsv_lmhead_argmax_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
+    lib.jsv_lmhead_argmax_noalloc.restype = ctypes.c_int
     lib.jsv_kernel_launches.argtypes = []
     lib.jsv_kernel_launches.restype = ctypes.c_uint64
     _lib = lib
@@ -147,6 +153,14 @@ def jsv_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, workspace, workspac
                                   _addr(max_logit), _addr(workspace), int(workspace_bytes),
                                   _stream(stream))
     _check("jsv_lmhead_argmax", st)
+
+
+def jsv_lmhead_argmax_noalloc(hidden, w, T, d, V, argmax, max_logit, stream=None) -> None:
+    """LM-head argmax with the library's fixed scratch (no workspace, no
+    allocation); see include/jsv.h for its limits and sharing rules."""
+    st = load().jsv_lmhead_argmax_noalloc(_addr(hidden), _addr(w), int(T), int(d), int(V),
+                                          _addr(argmax), _addr(max_logit), _stream(stream))
+    _check("jsv_lmhead_argmax_noalloc", st)
 
 
 def jsv_accept_path(batch, tokens, argmax, max_path, path, accept_len, bonus, stream=None) -> None:
