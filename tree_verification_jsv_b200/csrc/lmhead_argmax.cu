@@ -1,18 +1,40 @@
-// LM-head projection fused with top-1 argmax.
+// LM-head projection fused with top-1 argmax, on tcgen05 tensor cores.
 //
 // JetSpec README, "JetSpec / Overview": the accepted path follows the
-// target's own logits; every reported run is greedy (temperature 0), so
-// each node needs only argmax_v <hidden[t], w[v]>.  Logits are reduced in
-// registers / shared memory and never written to memory.
+// target's own logits, and every reported run is greedy (temperature 0), so
+// each node needs only argmax_v <hidden[t], w[v]>.  Logits live in TMEM and
+// registers only; they are never written to memory.
 //
-// Cross-CTA reduction: each CTA folds its best (value, index) per node into
-// one 64-bit key with atomicMax.  The high word is the fp32 value mapped to
-// an order-preserving unsigned integer, the low word is ~index, so the
-// maximum key carries the largest value and, among equal values, the
+// Shape of the contraction: logits^T[v][t] = W[v][:] . H[t][:].  The
+// vocabulary is the MMA M dimension (128 rows per tile, operand A = W) and
+// the tree nodes are the N dimension (operand B = H), so a 64-node tree
+// still fills M = 128 and W -- the dominant byte stream -- is read exactly
+// once when T <= 512.
+//
+// Persistent kernel, one CTA per SM, 6 warps:
+//   warp 0      TMA producer: W tile (16-row boxes) + H tile per 64-wide K
+//               chunk into a ring of shared-memory stages
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator, per-column argmax
+//               across the 128 vocabulary rows (a transposing butterfly of
+//               64-bit keys), then one atomicMax per node
+// Each CTA owns a contiguous, balanced vocabulary range [V*c/G, V*(c+1)/G)
+// and walks it in 128-row tiles; the ragged last tile of a range loads only
+// the 16-row boxes it needs, so no SM gets a whole extra tile of bytes.
+// With T <= 256 nodes two accumulators alternate in TMEM so the epilogue of
+// one tile overlaps the main loop of the next; larger trees are processed in
+// groups of 512 nodes (two N = 256 MMAs per K step, one accumulator).
+//
+// Cross-CTA reduction: a 64-bit key per node whose high word is the fp32
+// value mapped to an order-preserving unsigned integer and whose low word is
+// ~index; atomicMax keeps the largest value and, among equal values, the
 // smallest index.
 #include "jsv_internal.cuh"
+#include "sm100.cuh"
 
 namespace jsv {
+
+using namespace sm100;
 
 __device__ __forceinline__ unsigned long long argmax_key(float f, int v) {
     if (f == 0.0f) f = 0.0f;                       // -0 and +0 compare equal
@@ -27,6 +49,10 @@ __device__ __forceinline__ float key_value(unsigned long long k) {
     return __uint_as_float(u);
 }
 
+__device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
+    return a > b ? a : b;
+}
+
 __global__ void argmax_finalize_kernel(const unsigned long long *__restrict__ keys, int T,
                                        int32_t *__restrict__ argmax, float *__restrict__ max_logit) {
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -36,68 +62,246 @@ __global__ void argmax_finalize_kernel(const unsigned long long *__restrict__ ke
     if (max_logit) max_logit[t] = key_value(k);
 }
 
-// ---------------------------------------------------------------------------
-// SIMT tile: 64 vocabulary rows x 64 nodes per CTA, 4x4 outputs per thread.
-// ---------------------------------------------------------------------------
-constexpr int kTV = 64, kTT = 64, kTK = 32;
+constexpr int kThreads = 192;
+constexpr int kMaxStages = 8;
+constexpr int kTileM = 128;
+constexpr int kBoxRowsW = 16;
+constexpr int kKChunk = 64;                  // bf16 elements per 128-B swizzle line
+constexpr uint32_t kStageA = kTileM * 128;   // 16 KB
+constexpr int kSmemBudget = 200 * 1024;      // ring of stages (dynamic smem)
 
-__global__ void __launch_bounds__(256)
-lmhead_argmax_simt_kernel(const uint16_t *__restrict__ H, const uint16_t *__restrict__ W,
-                          int T, int d, int V, unsigned long long *__restrict__ keys) {
-    __shared__ float Ws[kTK][kTV + 4];
-    __shared__ float Hs[kTK][kTT + 4];
-    __shared__ unsigned long long red[16][kTT];
-    const int v0 = blockIdx.x * kTV, t0 = blockIdx.y * kTT;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+struct LmParams {
+    int T, d, V;
+    int kchunks;       // d / 64
+    int ngroups;       // node groups
+    int group_nodes;   // nodes per group (<= 256 with 2 accumulators, else 512)
+    int box_rows;      // H box height (<= 256)
+    int max_sub;       // H boxes per stage (1 or 2)
+    int n_acc;         // accumulator buffers in TMEM (2 or 1)
+    int stages;
+    uint32_t stage_bytes;
+    unsigned long long *keys;
+    int32_t *status;
+};
 
-    for (int k0 = 0; k0 < d; k0 += kTK) {
-        for (int e = threadIdx.x; e < kTV * kTK; e += 256) {
-            const int r = e / kTK, kk = e % kTK, v = v0 + r;
-            Ws[kk][r] = v < V ? bf16_bits_to_float(W[(size_t)v * d + k0 + kk]) : 0.f;
+__device__ __forceinline__ void set_abort(volatile int *abort, int32_t *status) {
+    *abort = 1;
+    if (status) atomicCAS(status, 0, JSV_ERR_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmW16,
+                        const __grid_constant__ CUtensorMap tmH, const LmParams p) {
+    extern __shared__ uint8_t dsmem[];
+    __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t accf_bar[2], acce_bar[2], drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile int abort_sh;
+    __shared__ volatile int ep_fail;
+    __shared__ unsigned long long red[4][512];
+
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = gridDim.x, cta = blockIdx.x;
+    const int r0 = (int)((long long)p.V * cta / G), r1 = (int)((long long)p.V * (cta + 1) / G);
+    const int ntiles = (r1 - r0 + kTileM - 1) / kTileM;
+    const int items = ntiles * p.ngroups;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
         }
-        for (int e = threadIdx.x; e < kTT * kTK; e += 256) {
-            const int r = e / kTK, kk = e % kTK, t = t0 + r;
-            Hs[kk][r] = t < T ? bf16_bits_to_float(H[(size_t)t * d + k0 + kk]) : 0.f;
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&accf_bar[a], 1);
+            mbar_init(&acce_bar[a], 4);
         }
-        __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < kTK; ++kk) {
-            float av[4], bv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) av[i] = Ws[kk][ty * 4 + i];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) bv[j] = Hs[kk][tx * 4 + j];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-        }
-        __syncthreads();
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        ep_fail = 0;
+        fence_barrier_init();
     }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        unsigned long long best = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int v = v0 + ty * 4 + i;
-            if (v < V) {
-                const unsigned long long k = argmax_key(acc[i][j], v);
-                best = k > best ? k : best;
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmW);
+        prefetch_tensormap(&tmW16);
+        prefetch_tensormap(&tmH);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint64_t pol_w = policy_evict_first();
+            const uint64_t pol_h = policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            for (int it = 0; it < items && !abort_sh; ++it) {
+                const int vt = it / p.ngroups, g = it % p.ngroups;
+                const int row0 = r0 + vt * kTileM;
+                const int rows = min(kTileM, r1 - row0);
+                const int nbx = rows == kTileM ? 1 : (rows + kBoxRowsW - 1) / kBoxRowsW;
+                const int node0 = g * p.group_nodes;
+                const int in_group = min(p.group_nodes, p.T - node0);
+                const int nsub = in_group > 256 ? 2 : 1;
+                const uint32_t tx = (rows == kTileM ? kStageA : (uint32_t)nbx * (kBoxRowsW * 128)) +
+                                    (uint32_t)nsub * p.box_rows * 128;
+                bool ok = true;
+                for (int kc = 0; kc < p.kchunks; ++kc) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh)) {
+                        set_abort(&abort_sh, p.status);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = smem + (size_t)stage * p.stage_bytes;
+                    uint8_t *sb = sa + kStageA;
+                    mbar_arrive_expect_tx(&full_bar[stage], tx);
+                    if (rows == kTileM) {
+                        tma_load_2d_hint(sa, &tmW, &full_bar[stage], kc * kKChunk, row0, pol_w);
+                    } else {
+                        for (int bx = 0; bx < nbx; ++bx)
+                            tma_load_2d_hint(sa + bx * (kBoxRowsW * 128), &tmW16, &full_bar[stage],
+                                             kc * kKChunk, row0 + bx * kBoxRowsW, pol_w);
+                    }
+                    for (int s = 0; s < nsub; ++s)
+                        tma_load_2d_hint(sb + s * p.box_rows * 128, &tmH, &full_bar[stage], kc * kKChunk,
+                                         node0 + s * 256, pol_h);
+                    ++issued;
+                    if (++stage == p.stages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+            }
+            if (abort_sh) {
+                // let every load still in flight land before the CTA exits
+                int zero = 0;
+                const long long back = issued < p.stages ? issued : p.stages;
+                int s = stage;
+                uint32_t ph = phase;
+                for (long long i = 0; i < back; ++i) {
+                    if (s == 0) { s = p.stages; ph ^= 1; }
+                    --s;
+                    mbar_wait(&full_bar[s], ph, (volatile int *)&zero);
+                }
             }
         }
-        red[ty][tx * 4 + j] = best;
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int it = 0; it < items && !abort_sh; ++it) {
+                const int acc = it % p.n_acc;
+                const uint32_t use = (uint32_t)(it / p.n_acc);
+                if (!mbar_wait(&acce_bar[acc], (use & 1) ^ 1, &abort_sh)) {
+                    set_abort(&abort_sh, p.status);
+                    break;
+                }
+                tc_fence_after();
+                const int g = it % p.ngroups;
+                const int node0 = g * p.group_nodes;
+                const int in_group = min(p.group_nodes, p.T - node0);
+                const int n0 = min(256, (in_group + 15) & ~15);
+                const int n1 = in_group > 256 ? ((in_group - 256 + 15) & ~15) : 0;
+                const uint32_t id0 = idesc_bf16_f32(kTileM, n0, false, false);
+                const uint32_t id1 = idesc_bf16_f32(kTileM, n1 > 0 ? n1 : 16, false, false);
+                const uint32_t d0 = tmem + (uint32_t)acc * 256u;
+                bool ok = true;
+                for (int kc = 0; kc < p.kchunks; ++kc) {
+                    if (!mbar_wait(&full_bar[stage], phase, &abort_sh)) {
+                        set_abort(&abort_sh, p.status);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_addr(smem + (size_t)stage * p.stage_bytes);
+                    const uint32_t sb = sa + kStageA;
+#pragma unroll
+                    for (int kk = 0; kk < kKChunk / 16; ++kk) {
+                        const uint32_t accum = (kc | kk) != 0;
+                        mma_bf16_ss(d0, desc_kmajor_sw128(sa + kk * 32), desc_kmajor_sw128(sb + kk * 32), id0,
+                                    accum);
+                        if (n1)
+                            mma_bf16_ss(d0 + 256, desc_kmajor_sw128(sa + kk * 32),
+                                        desc_kmajor_sw128(sb + p.box_rows * 128 + kk * 32), id1, accum);
+                    }
+                    mma_commit(&empty_bar[stage]);
+                    if (++stage == p.stages) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                mma_commit(&accf_bar[acc]);
+            }
+            // every MMA issued above has finished before TMEM is released
+            int zero = 0;
+            mma_commit(&drain_bar);
+            mbar_wait(&drain_bar, 0, (volatile int *)&zero);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 2;
+        const int sub = warp & 3;                    // TMEM lanes this warp may access
+        const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
+        const int et = threadIdx.x - 64;
+        for (int it = 0; it < items; ++it) {
+            const int acc = it % p.n_acc;
+            const uint32_t use = (uint32_t)(it / p.n_acc);
+            if (!mbar_wait(&accf_bar[acc], use & 1, &abort_sh)) {
+                set_abort(&abort_sh, p.status);
+                ep_fail = 1;
+            }
+            named_barrier(1, 128);
+            if (ep_fail) break;
+            tc_fence_after();
+            const int vt = it / p.ngroups, g = it % p.ngroups;
+            const int v = r0 + vt * kTileM + sub * 32 + lane;
+            const bool vvalid = v < r1;
+            const int node0 = g * p.group_nodes;
+            const int in_group = min(p.group_nodes, p.T - node0);
+            const int ncols = (in_group + 31) & ~31;
+            for (int c0 = 0; c0 < ncols; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)acc * 256u + (uint32_t)c0, r);
+                tmem_ld_wait();
+                unsigned long long x[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    x[j] = (vvalid && c0 + j < in_group) ? argmax_key(__uint_as_float(r[j]), v) : 0ull;
+                // transposing butterfly: afterwards lane l holds column c0 + l
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+                    const bool upper = (lane & o) != 0;
+#pragma unroll
+                    for (int i = 0; i < o; ++i) {
+                        const unsigned long long send = upper ? x[i] : x[i + o];
+                        const unsigned long long keep = upper ? x[i + o] : x[i];
+                        x[i] = umax64(keep, __shfl_xor_sync(0xffffffffu, send, o));
+                    }
+                }
+                red[ew][c0 + lane] = x[0];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acce_bar[acc]);
+            named_barrier(1, 128);
+            for (int c = et; c < in_group; c += 128) {
+                const unsigned long long k = umax64(umax64(red[0][c], red[1][c]), umax64(red[2][c], red[3][c]));
+                if (k) atomicMax(&p.keys[node0 + c], k);
+            }
+            named_barrier(1, 128);
+        }
     }
+
+    tc_fence_before();
     __syncthreads();
-    if (threadIdx.x < kTT) {
-        unsigned long long best = 0;
-        for (int y = 0; y < 16; ++y) best = red[y][threadIdx.x] > best ? red[y][threadIdx.x] : best;
-        const int t = t0 + threadIdx.x;
-        if (t < T && best) atomicMax(&keys[t], best);
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -108,11 +312,55 @@ size_t lmhead_workspace_bytes(int T, int d, int V) {
 
 cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int T, int d, int V,
                                  int32_t *argmax, float *max_logit, void *ws, cudaStream_t st) {
+    int32_t *status = nullptr;
     auto *keys = static_cast<unsigned long long *>(ws);
+    LmParams p;
+    p.T = T; p.d = d; p.V = V;
+    p.kchunks = d / kKChunk;
+    if (T <= 256) {
+        p.group_nodes = (T + 15) & ~15;
+        p.box_rows = p.group_nodes;
+        p.ngroups = 1;
+        p.max_sub = 1;
+        p.n_acc = 2;
+    } else {
+        p.group_nodes = 512;
+        p.box_rows = 256;
+        p.ngroups = (T + 511) / 512;
+        p.max_sub = 2;
+        p.n_acc = 1;
+    }
+    p.stage_bytes = kStageA + (uint32_t)p.max_sub * p.box_rows * 128;
+    p.stages = kSmemBudget / (int)p.stage_bytes;
+    if (p.stages > kMaxStages) p.stages = kMaxStages;
+    p.keys = keys;
+    p.status = status;
+
+    CUtensorMap tmW, tmW16, tmH;
+    if (!encode_tensor_map_2d(&tmW, w, (uint64_t)d, (uint64_t)V, (uint64_t)d * 2, kKChunk, kTileM))
+        return cudaErrorInvalidValue;
+    if (!encode_tensor_map_2d(&tmW16, w, (uint64_t)d, (uint64_t)V, (uint64_t)d * 2, kKChunk, kBoxRowsW))
+        return cudaErrorInvalidValue;
+    if (!encode_tensor_map_2d(&tmH, hidden, (uint64_t)d, (uint64_t)T, (uint64_t)d * 2, kKChunk, p.box_rows))
+        return cudaErrorInvalidValue;
+
+    const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(lmhead_argmax_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemBudget + 1024);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
     cudaError_t e = cudaMemsetAsync(keys, 0, (size_t)T * sizeof(unsigned long long), st);
     if (e != cudaSuccess) return e;
-    dim3 grid((V + kTV - 1) / kTV, (T + kTT - 1) / kTT);
-    lmhead_argmax_simt_kernel<<<grid, 256, 0, st>>>(hidden, w, T, d, V, keys);
+    const int tiles = (V + kTileM - 1) / kTileM;
+    int grid = device_sm_count();
+    if (grid <= 0) return cudaErrorInvalidDevice;
+    if (grid > tiles) grid = tiles;
+    lmhead_argmax_tc_kernel<<<grid, kThreads, smem, st>>>(tmW, tmW16, tmH, p);
     argmax_finalize_kernel<<<(T + 255) / 256, 256, 0, st>>>(keys, T, argmax, max_logit);
     count_launches(2);
     return cudaGetLastError();
