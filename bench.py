@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--workload", default="8b_64", choices=list(DESCRIPTION))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile", choices=["attention", "lmhead", "accept", "compact"],
+                    help="run only this call K times after W warm-up (for ncu); prints its mean time")
     return ap.parse_args()
 
 
@@ -158,19 +160,19 @@ def source_sha(*files):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key, workload, launches_units):
-    """DRAM bytes per launch from the committed ncu summary, if its source
-    hash still matches the kernel source (else None)."""
+def ncu_traffic(kernel_key, workload):
+    """DRAM bytes per launch (read + write) of the dominant kernel from the
+    committed ncu summary -- only for the workload it was captured on and only
+    while the kernel's source hash still matches (else None)."""
     p = ROOT / "profiles" / "ncu_traffic.json"
     if not p.exists():
         return None
     d = json.loads(p.read_text()).get(kernel_key)
-    if not d:
+    if not d or d.get("workload") != workload:
         return None
     if d.get("source_sha") != source_sha(*d["sources"]):
         return None
-    per_unit = d["dram_bytes_per_launch"] / d["units_per_launch"]
-    return int(round(per_unit * launches_units))
+    return int(d["dram_bytes_per_launch"])
 
 
 # ---------------------------------------------------------------------------
@@ -260,6 +262,22 @@ def run_gpu(args, rank, world, local_rank):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=f"cuda:{local_rank}")
     stream = torch.cuda.current_stream()
 
+    if args.profile:
+        call = getattr(st, args.profile)
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert int(st.status.item()) == 0
+        print(json.dumps({"profile": args.profile, "workload": args.workload,
+                          "mean_us_warm_l2": 1e3 * e0.elapsed_time(e1) / args.steps}), flush=True)
+        return
+
     # correctness of this very launch configuration against stored oracle values
     st.run()
     torch.cuda.synchronize()
@@ -345,7 +363,7 @@ def run_gpu(args, rank, world, local_rank):
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"
     roof["algorithmic_bytes_per_launch"] = m["bytes"]
     roof["algorithmic_flops_per_launch"] = m["flops"]
-    roof["traffic"] = ncu_traffic(dom, args.workload, m["bytes"])
+    roof["traffic"] = ncu_traffic(dom, args.workload)
 
     value = world * wl.T / (step_ms_max * 1e-3)
     line = {

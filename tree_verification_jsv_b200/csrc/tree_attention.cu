@@ -1,123 +1,466 @@
-// Tree-causal attention over a paged KV prefix, split-KV.
+// Tree-causal attention over a paged KV prefix on tcgen05 tensor cores.
 //
 // JetSpec README, "JetSpec / Overview": the whole draft tree is verified in
 // one forward pass under a tree-causal mask.  Node i of request b attends to
 // prefix slots [0, P) and to slot P + j for every ancestor-or-self j of i.
-// The prefix is cut into S splits processed by separate CTAs; the tree part
-// rides with the last split; a combine pass merges the (max, sum, output)
-// partials with the usual log-sum-exp rescaling.
 //
-// SIMT version: one warp per (node, query head, split); each lane owns D/32
-// output dimensions.
+// Work decomposition (one CTA per unit):
+//   (request b, KV head g, M-tile of 128 query rows, KV split s)
+// Query rows of (b, g) pack the G = Hq/Hkv heads that share KV head g:
+// row r <-> node r / G, head g*G + r % G, so every K/V tile loaded serves
+// G*128/G = 128 query rows (GQA packing).  The prefix is cut into 128-key
+// tiles that start on page boundaries; split s takes a contiguous run of
+// them, and the last split also takes the tree tiles, which cover slots
+// [P & ~15, P + N) and apply the ancestor mask.  Each split writes an
+// unnormalised fp32 partial (O, row max, row sum); a small combine kernel
+// merges the splits with log-sum-exp rescaling and rounds to bf16.
+//
+// Per CTA, 6 warps:
+//   warp 0      TMA producer: K and V of each 128-key tile, one 16-slot
+//               page x 64-dim box per copy, into a 2-stage ring
+//   warp 1      TMEM allocator and single-thread MMA issuer:
+//               S_j = Q K_j^T into one of two TMEM S buffers, then
+//               O += P_{j-1} V_{j-1} once softmax has written P_{j-1}
+//   warps 2..5  softmax: one query row per thread; load S_j from TMEM,
+//               mask, online softmax in the log2 domain, write P_j (bf16)
+//               to shared memory; rescale O in TMEM only when the running
+//               max grows by more than 8 (2^8), which keeps exp2 arguments
+//               bounded without touching O on most tiles
+// Shared memory: Q (16 KB per 64 dims), P (32 KB), 2 x (K, V) stages.
 #include "jsv_internal.cuh"
+#include "sm100.cuh"
 
 #include <math.h>
 
 namespace jsv {
 
-constexpr int kAttnWarps = 8;
+using namespace sm100;
 
-static int attention_splits(const BatchArgs &a) {
-    int s = (a.max_prefix + 511) / 512;
-    return s < 1 ? 1 : (s > 16 ? 16 : s);
+constexpr int kAttnThreads = 192;
+constexpr int kKeyTile = 128;
+constexpr int kRowsPerCta = 128;
+constexpr int kStages = 2;
+constexpr int kMaxTreeWords = 16;          // 512 nodes
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
-size_t attention_workspace_bytes(const BatchArgs &a) {
-    const size_t rows = (size_t)a.total_nodes * a.Hq;
-    return (size_t)attention_splits(a) * rows * ((size_t)a.D + 2) * sizeof(float);
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Ancestor-or-self bitset of request-local node i: lane w holds bits
-// [32w, 32w + 32).  Returns false if the parent chain is malformed.
-__device__ __forceinline__ bool ancestor_bits(const BatchArgs &a, const Request &r, int i,
-                                              int lane, unsigned &bits) {
-    bits = 0;
-    int j = i, steps = 0;
-    while (j != -1) {
-        if (steps++ > r.n) return false;
-        if ((j >> 5) == lane) bits |= 1u << (j & 31);
-        const int p = a.parent[r.base + j];
-        if (j == 0 ? p != -1 : (p < 0 || p >= j)) return false;
-        j = p;
-    }
-    return true;
+struct AttnParams {
+    BatchArgs a;
+    const uint16_t *q;
+    float scale_log2;
+    int S;                 // splits
+    float *ws_o;           // [S][T*Hq][D]
+    float *ws_ml;          // [S][T*Hq][2]
+};
+
+template <int D>
+struct AttnSmem {
+    static constexpr int kQBytes = kRowsPerCta * D * 2;        // Q tile
+    static constexpr int kPBytes = kRowsPerCta * kKeyTile * 2;  // P tile (32 KB)
+    static constexpr int kKVBytes = kKeyTile * D * 2;          // one K (or V) tile
+    static constexpr int kStageBytes = 2 * kKVBytes;
+    static constexpr int kTotal = kQBytes + kPBytes + kStages * kStageBytes;
+};
+
+// Byte offset of 16-byte chunk `c` of row `r` in a K-major SW128 operand
+// region (rows of 128 B, 8-row atoms; chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
+    return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttnWarps * 32)
-tree_attention_simt_kernel(BatchArgs a, const uint16_t *__restrict__ q,
-                           const uint16_t *__restrict__ kc, const uint16_t *__restrict__ vc,
-                           float scale_log2, int S, float *__restrict__ ws_o,
-                           float *__restrict__ ws_ml) {
-    constexpr int DPL = D / 32;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(kAttnThreads, 1)
+tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                         const AttnParams prm) {
+    using L = AttnSmem<D>;
+    constexpr int kHalves = D / 64;
+    extern __shared__ uint8_t dsmem[];
+    __shared__ __align__(8) uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+    __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full, o_done, q_ready, drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile int abort_sh;
+    __shared__ volatile int sm_fail;
+    __shared__ uint32_t anc[kRowsPerCta][kMaxTreeWords];
+
+    const BatchArgs &a = prm.a;
     const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
     const int G = a.Hq / a.Hkv;
-    const int rloc = blockIdx.x * kAttnWarps + warp;
     const int split = blockIdx.y;
+    const int m0 = blockIdx.x * kRowsPerCta;
+
+    // request geometry (uniform per CTA); invalid requests are flagged and skipped
     Request r;
     if (!load_request(a, b, r)) return;
-    if (rloc >= r.n * G) return;
-    const int i = rloc / G, h = g * G + rloc % G, t = r.base + i;
-    unsigned anc;
-    if (!ancestor_bits(a, r, i, lane, anc)) {
-        if (lane == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
-        return;
+    const int rows_total = r.n * G;
+    if (m0 >= rows_total) return;
+    const int rows_here = min(kRowsPerCta, rows_total - m0);
+
+    // tile schedule for this split
+    const int prefix_tiles = (r.P + kKeyTile - 1) / kKeyTile;
+    const int t_begin = (int)((long long)prefix_tiles * split / prm.S);
+    const int t_end = (int)((long long)prefix_tiles * (split + 1) / prm.S);
+    const int P0 = r.P & ~15;                    // tree tiles start on a page boundary
+    const int tree_tiles = (split == prm.S - 1) ? (r.P + r.n - P0 + kKeyTile - 1) / kKeyTile : 0;
+    const int ntiles = (t_end - t_begin) + tree_tiles;
+
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;
+    uint8_t *sP = smem + L::kQBytes;
+    uint8_t *sKV = sP + L::kPBytes;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], 4);
+        }
+        mbar_init(&p_full, 4);
+        mbar_init(&o_done, 1);
+        mbar_init(&q_ready, 4);
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        sm_fail = 0;
+        fence_barrier_init();
     }
-    float qv[DPL];
-    const uint16_t *qp = q + ((size_t)t * a.Hq + h) * D + lane * DPL;
-#pragma unroll
-    for (int x = 0; x < DPL; ++x) qv[x] = bf16_bits_to_float(qp[x]) * scale_log2;
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+    const uint32_t tS = tmem;              // S buffers: columns [0,128) and [128,256)
+    const uint32_t tO = tmem + 256;        // O: columns [256, 256 + D)
 
-    float m = -INFINITY, l = 0.f, o[DPL];
-#pragma unroll
-    for (int x = 0; x < DPL; ++x) o[x] = 0.f;
-
-    auto visit = [&](int slot) {
-        const long long row = slot_phys_row(a, b, slot);
-        if (row < 0) return;
-        const size_t off = ((size_t)row * a.Hkv + g) * D + lane * DPL;
-        float part = 0.f;
-#pragma unroll
-        for (int x = 0; x < DPL; ++x) part = fmaf(qv[x], bf16_bits_to_float(kc[off + x]), part);
-#pragma unroll
-        for (int sh = 16; sh > 0; sh >>= 1) part += __shfl_xor_sync(0xffffffffu, part, sh);
-        const float mn = fmaxf(m, part);
-        const float c = exp2f(m - mn), p = exp2f(part - mn);
-        l = l * c + p;
-#pragma unroll
-        for (int x = 0; x < DPL; ++x) o[x] = fmaf(p, bf16_bits_to_float(vc[off + x]), o[x] * c);
-        m = mn;
+    // logical tile index -> first logical slot
+    auto tile_slot0 = [&](int j) -> int {
+        return j < (t_end - t_begin) ? (t_begin + j) * kKeyTile : P0 + (j - (t_end - t_begin)) * kKeyTile;
     };
 
-    const int lo = (int)((long long)r.P * split / S), hi = (int)((long long)r.P * (split + 1) / S);
-    for (int s = lo; s < hi; ++s) visit(s);
-    if (split == S - 1) {
-        for (int j = 0; j < r.n; ++j) {
-            const unsigned w = __shfl_sync(0xffffffffu, anc, j >> 5);
-            if ((w >> (j & 31)) & 1u) visit(r.P + j);
+    if (warp == 0) {
+        // ----------------------------------------------------------- producer
+        if (lane == 0 && ntiles > 0) {
+            prefetch_tensormap(&tmK);
+            prefetch_tensormap(&tmV);
+            const int oob = a.num_pages * a.page_size;   // fully out-of-bounds slot coordinate
+            const int mapped_pages = (r.P + r.n + a.page_size - 1) / a.page_size;
+            long long issued = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int j = 0; j < ntiles && !abort_sh; ++j) {
+                if (!mbar_wait(&kv_empty[stage], phase ^ 1, &abort_sh)) {
+                    abort_sh = 1;
+                    flag_error(a.dev_status, JSV_ERR_TIMEOUT);
+                    break;
+                }
+                uint8_t *sK = sKV + stage * L::kStageBytes;
+                uint8_t *sV = sK + L::kKVBytes;
+                const int slot0 = tile_slot0(j);
+                mbar_arrive_expect_tx(&k_full[stage], L::kKVBytes);
+                mbar_arrive_expect_tx(&v_full[stage], L::kKVBytes);
+                for (int pg = 0; pg < kKeyTile / 16; ++pg) {
+                    const int lp = slot0 / 16 + pg;          // logical page
+                    int z = oob;
+                    if (lp < mapped_pages) {
+                        const int page = a.page_table[(size_t)b * a.max_pages_per_req + lp];
+                        if (page >= 0 && page < a.num_pages) z = page * a.page_size;
+                        else flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+                    }
+                    for (int h = 0; h < kHalves; ++h) {
+                        tma_load_3d(sK + h * (kKeyTile * 128) + pg * 2048, &tmK, &k_full[stage], h * 64, g, z);
+                        tma_load_3d(sV + h * (kKeyTile * 128) + pg * 2048, &tmV, &v_full[stage], h * 64, g, z);
+                    }
+                }
+                ++issued;
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
+            }
+            if (abort_sh) {
+                int zero = 0;
+                const long long back = issued < kStages ? issued : kStages;
+                int s = stage;
+                uint32_t ph = phase;
+                for (long long i = 0; i < back; ++i) {
+                    if (s == 0) { s = kStages; ph ^= 1; }
+                    --s;
+                    mbar_wait(&k_full[s], ph, (volatile int *)&zero);
+                    mbar_wait(&v_full[s], ph, (volatile int *)&zero);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer
+        if (lane == 0 && ntiles > 0) {
+            const uint32_t id_s = idesc_bf16_f32(128, kKeyTile, false, false);
+            const uint32_t id_o = idesc_bf16_f32(128, D, false, true);
+            const uint32_t aQ = smem_addr(sQ), aP = smem_addr(sP);
+            bool ok = mbar_wait(&q_ready, 0, &abort_sh);
+            int kst = 0;                 // stage of tile j
+            uint32_t kph = 0;
+            int vst = 0;                 // stage of tile j-1 (for PV)
+            uint32_t vph = 0;
+            for (int j = 0; ok && j <= ntiles; ++j) {
+                if (j < ntiles) {
+                    // S_j = Q K_j^T into buffer j % 2
+                    const int sb = j & 1;
+                    ok = mbar_wait(&k_full[kst], kph, &abort_sh) &&
+                         mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, &abort_sh);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t aK = smem_addr(sKV + kst * L::kStageBytes);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * (kRowsPerCta * 128) + (kk & 3) * 32;
+                        const uint32_t offk = (kk >> 2) * (kKeyTile * 128) + (kk & 3) * 32;
+                        mma_bf16_ss(tS + sb * 128, desc_kmajor_sw128(aQ + off), desc_kmajor_sw128(aK + offk), id_s,
+                                    kk > 0);
+                    }
+                    mma_commit(&s_full[sb]);
+                    if (++kst == kStages) { kst = 0; kph ^= 1; }
+                }
+                if (j >= 1) {
+                    // O += P_{j-1} V_{j-1}
+                    const int jj = j - 1;
+                    ok = mbar_wait(&p_full, jj & 1, &abort_sh) && mbar_wait(&v_full[vst], vph, &abort_sh);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t aV = smem_addr(sKV + vst * L::kStageBytes + L::kKVBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kKeyTile / 16; ++kk) {
+                        const uint32_t offp = (kk >> 2) * (kRowsPerCta * 128) + (kk & 3) * 32;
+                        // V is MN-major: 16 keys = 16 lines of 128 B; 64-dim blocks 16 KB apart
+                        mma_bf16_ss(tO, desc_kmajor_sw128(aP + offp),
+                                    desc_mnmajor_sw128(aV + kk * 2048, kKeyTile * 128, 1024), id_o,
+                                    (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&o_done);
+                    mma_commit(&kv_empty[vst]);
+                    if (++vst == kStages) { vst = 0; vph ^= 1; }
+                }
+            }
+            if (!ok) {
+                abort_sh = 1;
+                flag_error(a.dev_status, JSV_ERR_TIMEOUT);
+            }
+            int zero = 0;
+            mma_commit(&drain_bar);
+            mbar_wait(&drain_bar, 0, (volatile int *)&zero);
+        }
+    } else {
+        // ----------------------------------------------------------- softmax
+        const int sub = warp & 3;
+        const int row = sub * 32 + lane;            // TMEM lane == query row in the tile
+        const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
+        const int et = threadIdx.x - 64;             // 0..127
+        const bool row_valid = row < rows_here;
+        const int rg = m0 + row;                     // row within (b, g)
+        const int node = rg / G;                     // request-local node
+        const int head = g * G + rg % G;
+
+        // Q tile: rows x D bf16 into the K-major SW128 layout (zero rows past the end)
+        for (int e = et; e < kRowsPerCta * (D / 8); e += 128) {
+            const int rr = e / (D / 8), c = e % (D / 8);
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (rr < rows_here) {
+                const int rgg = m0 + rr;
+                const uint16_t *src = prm.q + ((size_t)(r.base + rgg / G) * a.Hq + g * G + rgg % G) * D + c * 8;
+                v = *reinterpret_cast<const uint4 *>(src);
+            }
+            *reinterpret_cast<uint4 *>(sQ + (c >> 3) * (kRowsPerCta * 128) + sw128_offset(rr, c & 7)) = v;
+        }
+        // ancestor-or-self bitsets of this tile's rows (only the last split uses them)
+        if (tree_tiles > 0 && row_valid) {
+            for (int w = 0; w < kMaxTreeWords; ++w) anc[row][w] = 0;
+            int j = node, steps = 0;
+            while (j != -1) {
+                if (steps++ > r.n || j >= 32 * kMaxTreeWords) { sm_fail = 1; break; }
+                anc[row][j >> 5] |= 1u << (j & 31);
+                const int p = a.parent[r.base + j];
+                if (j == 0 ? p != -1 : (p < 0 || p >= j)) { sm_fail = 1; break; }
+                j = p;
+            }
+        }
+        fence_async_smem();
+        named_barrier(1, 128);
+        if (sm_fail) {
+            if (et == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_ready);
+
+        float m_used = -INFINITY, l = 0.f;
+        const float sl2 = prm.scale_log2;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j) {
+            const int sb = j & 1;
+            if (!mbar_wait(&s_full[sb], (j >> 1) & 1, &abort_sh)) ok = false;
+            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+            tc_fence_after();
+            const int slot0 = tile_slot0(j);
+            const bool is_tree = j >= (t_end - t_begin);
+            const bool full_tile = !is_tree && slot0 + kKeyTile <= r.P;
+            const uint32_t sbase = tS + sb * 128 + lane_addr;
+            // visibility of key column c of this tile for this row
+            auto visible = [&](int c) -> bool {
+                const int slot = slot0 + c;
+                if (!is_tree) return slot < r.P;
+                const int jn = slot - r.P;
+                return jn >= 0 && jn < r.n && row_valid &&
+                       ((anc[row][(jn >> 5) & (kMaxTreeWords - 1)] >> (jn & 31)) & 1u);
+            };
+            // pass 1: row max of the scaled, masked scores
+            float tmax = -INFINITY;
+#pragma unroll
+            for (int c0 = 0; c0 < kKeyTile; c0 += 32) {
+                uint32_t rr[32];
+                tmem_ld_32x32b_x32(sbase + c0, rr);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    const bool vis = full_tile || visible(c0 + x);
+                    tmax = fmaxf(tmax, vis ? __uint_as_float(rr[x]) * sl2 : -INFINITY);
+                }
+            }
+            // running max with a rescale threshold
+            float m_new = m_used;
+            if (tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY)) m_new = tmax;
+            const float corr = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);   // 0 when m_used = -inf
+            // pass 2: probabilities, their sum, and the packed bf16 row
+            float psum = 0.f;
+            uint32_t pk[kKeyTile / 2];
+#pragma unroll
+            for (int c0 = 0; c0 < kKeyTile; c0 += 32) {
+                uint32_t rr[32];
+                tmem_ld_32x32b_x32(sbase + c0, rr);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; x += 2) {
+                    float p0 = 0.f, p1 = 0.f;
+                    if (m_new != -INFINITY) {
+                        if (full_tile || visible(c0 + x)) p0 = fast_exp2(__uint_as_float(rr[x]) * sl2 - m_new);
+                        if (full_tile || visible(c0 + x + 1)) p1 = fast_exp2(__uint_as_float(rr[x + 1]) * sl2 - m_new);
+                    }
+                    psum += p0 + p1;
+                    pk[(c0 + x) / 2] = pack_bf16x2(p0, p1);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[sb]);
+            l = l * corr + psum;
+
+            // O and the P buffer are free once PV_{j-1} has completed
+            if (j >= 1) {
+                if (!mbar_wait(&o_done, (j - 1) & 1, &abort_sh)) ok = false;
+                if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, corr != 1.f)) {
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t ov[32];
+                        tmem_ld_32x32b_x32(tO + lane_addr + c0, ov);
+                        tmem_ld_wait();
+                        uint32_t lo[16], hi[16];
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            lo[x] = __float_as_uint(__uint_as_float(ov[x]) * corr);
+                            hi[x] = __float_as_uint(__uint_as_float(ov[16 + x]) * corr);
+                        }
+                        tmem_st_32x32b_x16(tO + lane_addr + c0, lo);
+                        tmem_st_32x32b_x16(tO + lane_addr + c0 + 16, hi);
+                    }
+                    tmem_st_wait();
+                }
+            }
+            m_used = m_new;
+            // P row (bf16) into the K-major SW128 layout: keys 0-63 and 64-127 in two regions
+#pragma unroll
+            for (int c = 0; c < kKeyTile / 8; ++c) {
+                const uint4 v = make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+                *reinterpret_cast<uint4 *>(sP + (c >> 3) * (kRowsPerCta * 128) + sw128_offset(row, c & 7)) = v;
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full);
+        }
+
+        // final partial: O (unnormalised), running max (log2 domain) and sum
+        float ofin[D];
+        bool have_o = ok && ntiles > 0;
+        if (have_o) {
+            if (!mbar_wait(&o_done, (ntiles - 1) & 1, &abort_sh)) ok = false;
+            if (__any_sync(0xffffffffu, !ok)) have_o = false;
+        }
+        if (have_o) {
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t rr[32];
+                tmem_ld_32x32b_x32(tO + lane_addr + c0, rr);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) ofin[c0 + x] = __uint_as_float(rr[x]);
+            }
+        } else {
+#pragma unroll
+            for (int x = 0; x < D; ++x) ofin[x] = 0.f;
+            m_used = -INFINITY;
+            l = 0.f;
+            if (!ok) {
+                abort_sh = 1;
+                flag_error(a.dev_status, JSV_ERR_TIMEOUT);
+            }
+        }
+        if (row_valid) {
+            const size_t rows = (size_t)a.total_nodes * a.Hq;
+            const size_t row_id = (size_t)(r.base + node) * a.Hq + head;
+            float4 *po = reinterpret_cast<float4 *>(prm.ws_o + ((size_t)split * rows + row_id) * D);
+#pragma unroll
+            for (int x = 0; x < D / 4; ++x) po[x] = make_float4(ofin[4 * x], ofin[4 * x + 1], ofin[4 * x + 2], ofin[4 * x + 3]);
+            prm.ws_ml[((size_t)split * rows + row_id) * 2 + 0] = m_used;
+            prm.ws_ml[((size_t)split * rows + row_id) * 2 + 1] = l;
         }
     }
-    const size_t row_id = (size_t)t * a.Hq + h;
-    const size_t rows = (size_t)a.total_nodes * a.Hq;
-    float *po = ws_o + ((size_t)split * rows + row_id) * D + lane * DPL;
-#pragma unroll
-    for (int x = 0; x < DPL; ++x) po[x] = o[x];
-    if (lane == 0) {
-        ws_ml[((size_t)split * rows + row_id) * 2 + 0] = m;
-        ws_ml[((size_t)split * rows + row_id) * 2 + 1] = l;
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
 }
 
+// ---------------------------------------------------------------------------
+// Split combine: one warp per (node, head) row.
+// ---------------------------------------------------------------------------
+constexpr int kCombineWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(kAttnWarps * 32)
+__global__ void __launch_bounds__(kCombineWarps * 32)
 tree_attention_combine_kernel(BatchArgs a, int S, const float *__restrict__ ws_o,
                               const float *__restrict__ ws_ml, uint16_t *__restrict__ out) {
     constexpr int DPL = D / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
     const int G = a.Hq / a.Hkv;
-    const int rloc = blockIdx.x * kAttnWarps + warp;
+    const int rloc = blockIdx.x * kCombineWarps + warp;
     Request r;
     if (!load_request(a, b, r)) return;
     if (rloc >= r.n * G) return;
@@ -150,28 +493,81 @@ tree_attention_combine_kernel(BatchArgs a, int S, const float *__restrict__ ws_o
     }
 }
 
-cudaError_t launch_tree_attention(const BatchArgs &a, const uint16_t *q, const uint16_t *k_cache,
-                                  const uint16_t *v_cache, float scale, uint16_t *out, void *ws,
-                                  cudaStream_t st) {
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static int attention_splits(const BatchArgs &a) {
+    // Split the prefix so the grid fills whole waves of SMs (1 CTA per SM),
+    // keeping at least two 128-key tiles per split.
+    const int G = a.Hq / a.Hkv;
+    const int mtiles = (a.max_nodes * G + kRowsPerCta - 1) / kRowsPerCta;
+    const long long units = (long long)a.B * a.Hkv * mtiles;
+    const int prefix_tiles = (a.max_prefix + kKeyTile - 1) / kKeyTile;
+    int cap = prefix_tiles / 2;
+    if (cap < 1) cap = 1;
+    if (cap > 32) cap = 32;
+    const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+    int best = 1;
+    double best_eff = -1.0;
+    for (int s = 1; s <= cap; ++s) {
+        const long long ctas = units * s;
+        const long long waves = (ctas + sms - 1) / sms;
+        const double eff = (double)ctas / (double)(waves * sms);
+        if (eff >= 0.9 && ctas >= sms) return s;
+        if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+    }
+    return best;
+}
+
+size_t attention_workspace_bytes(const BatchArgs &a) {
+    const size_t rows = (size_t)a.total_nodes * a.Hq;
+    return (size_t)attention_splits(a) * rows * ((size_t)a.D + 2) * sizeof(float);
+}
+
+template <int D>
+static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_t *k_cache,
+                            const uint16_t *v_cache, float scale, uint16_t *out, void *ws, cudaStream_t st) {
+    using Lt = AttnSmem<D>;
     const int S = attention_splits(a);
     const int G = a.Hq / a.Hkv;
     const size_t rows = (size_t)a.total_nodes * a.Hq;
-    float *ws_o = static_cast<float *>(ws);
-    float *ws_ml = ws_o + (size_t)S * rows * a.D;
-    const float scale_log2 = scale * 1.4426950408889634f;
-    dim3 grid((a.max_nodes * G + kAttnWarps - 1) / kAttnWarps, S, a.B * a.Hkv);
-    dim3 cgrid(grid.x, 1, grid.z);
-    if (a.D == 128) {
-        tree_attention_simt_kernel<128><<<grid, kAttnWarps * 32, 0, st>>>(a, q, k_cache, v_cache,
-                                                                          scale_log2, S, ws_o, ws_ml);
-        tree_attention_combine_kernel<128><<<cgrid, kAttnWarps * 32, 0, st>>>(a, S, ws_o, ws_ml, out);
-    } else {
-        tree_attention_simt_kernel<64><<<grid, kAttnWarps * 32, 0, st>>>(a, q, k_cache, v_cache,
-                                                                         scale_log2, S, ws_o, ws_ml);
-        tree_attention_combine_kernel<64><<<cgrid, kAttnWarps * 32, 0, st>>>(a, S, ws_o, ws_ml, out);
+    AttnParams prm;
+    prm.a = a;
+    prm.q = q;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.S = S;
+    prm.ws_o = static_cast<float *>(ws);
+    prm.ws_ml = prm.ws_o + (size_t)S * rows * D;
+
+    CUtensorMap tmK, tmV;
+    const uint64_t slots = (uint64_t)a.num_pages * a.page_size;
+    if (!encode_tensor_map_3d(&tmK, k_cache, D, a.Hkv, slots, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2, 64, 1, 16))
+        return cudaErrorInvalidValue;
+    if (!encode_tensor_map_3d(&tmV, v_cache, D, a.Hkv, slots, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2, 64, 1, 16))
+        return cudaErrorInvalidValue;
+    const size_t smem = (size_t)Lt::kTotal + 1024;
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(tree_attention_tc_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
     }
+    dim3 grid((a.max_nodes * G + kRowsPerCta - 1) / kRowsPerCta, S, a.B * a.Hkv);
+    tree_attention_tc_kernel<D><<<grid, kAttnThreads, smem, st>>>(tmK, tmV, prm);
+    dim3 cgrid((a.max_nodes * G + kCombineWarps - 1) / kCombineWarps, 1, a.B * a.Hkv);
+    tree_attention_combine_kernel<D><<<cgrid, kCombineWarps * 32, 0, st>>>(a, S, prm.ws_o, prm.ws_ml, out);
     count_launches(2);
     return cudaGetLastError();
+}
+
+cudaError_t launch_tree_attention(const BatchArgs &a, const uint16_t *q, const uint16_t *k_cache,
+                                  const uint16_t *v_cache, float scale, uint16_t *out, void *ws,
+                                  cudaStream_t st) {
+    if (a.D == 128) return launch_d<128>(a, q, k_cache, v_cache, scale, out, ws, st);
+    return launch_d<64>(a, q, k_cache, v_cache, scale, out, ws, st);
 }
 
 }  // namespace jsv
