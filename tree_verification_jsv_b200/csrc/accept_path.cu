@@ -11,22 +11,32 @@
 
 namespace jsv {
 
-__global__ void __launch_bounds__(128)
+constexpr int kWalkWarps = 4;
+constexpr int kWalkMaxNodes = 512;
+
+__global__ void __launch_bounds__(kWalkWarps * 32)
 accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
                    const int32_t *__restrict__ argmax, int max_path, int32_t *__restrict__ path,
                    int32_t *__restrict__ accept_len, int32_t *__restrict__ bonus) {
-    const int warps = blockDim.x >> 5;
-    const int b = blockIdx.x * warps + (threadIdx.x >> 5);
+    // the request's parent / token / target-choice arrays, staged once
+    __shared__ int32_t s_par[kWalkWarps][kWalkMaxNodes];
+    __shared__ int32_t s_tok[kWalkWarps][kWalkMaxNodes];
+    __shared__ int32_t s_arg[kWalkWarps][kWalkMaxNodes];
+    const int w = threadIdx.x >> 5;
+    const int b = blockIdx.x * kWalkWarps + w;
     const int lane = threadIdx.x & 31;
     if (b >= a.B) return;
     int32_t *row = path + (size_t)b * max_path;
 
     Request r;
-    bool ok = load_request(a, b, r);
+    bool ok = load_request(a, b, r) && r.n <= kWalkMaxNodes;
     if (ok) {
         bool bad = false;
         for (int j = lane; j < r.n; j += 32) {
-            int p = a.parent[r.base + j];
+            const int p = a.parent[r.base + j];
+            s_par[w][j] = p;
+            s_tok[w][j] = tokens[r.base + j];
+            s_arg[w][j] = argmax[r.base + j];
             bad |= (j == 0) ? (p != -1) : (p < 0 || p >= j);
         }
         if (__any_sync(0xffffffffu, bad)) {
@@ -39,14 +49,15 @@ accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
         if (lane == 0) { accept_len[b] = 0; bonus[b] = -1; }
         return;
     }
+    __syncwarp();
 
     int cur = 0, len = 1;
     while (true) {
-        const int want = argmax[r.base + cur];
+        const int want = s_arg[w][cur];
         int found = -1;
         for (int j0 = cur + 1; j0 < r.n; j0 += 32) {
             const int j = j0 + lane;
-            const bool m = j < r.n && a.parent[r.base + j] == cur && tokens[r.base + j] == want;
+            const bool m = j < r.n && s_par[w][j] == cur && s_tok[w][j] == want;
             const unsigned bal = __ballot_sync(0xffffffffu, m);
             if (bal) { found = j0 + __ffs(bal) - 1; break; }
         }
@@ -62,7 +73,7 @@ accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
     if (lane == 0) {
         row[0] = 0;
         accept_len[b] = len - 1;
-        bonus[b] = argmax[r.base + cur];
+        bonus[b] = s_arg[w][cur];
     }
     for (int k = len + lane; k < max_path; k += 32) row[k] = -1;
 }
@@ -70,9 +81,8 @@ accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
 cudaError_t launch_accept_path(const BatchArgs &a, const int32_t *tokens, const int32_t *argmax,
                                int max_path, int32_t *path, int32_t *accept_len, int32_t *bonus,
                                cudaStream_t st) {
-    const int warps = 4;
-    dim3 grid((a.B + warps - 1) / warps);
-    accept_path_kernel<<<grid, warps * 32, 0, st>>>(a, tokens, argmax, max_path, path, accept_len, bonus);
+    dim3 grid((a.B + kWalkWarps - 1) / kWalkWarps);
+    accept_path_kernel<<<grid, kWalkWarps * 32, 0, st>>>(a, tokens, argmax, max_path, path, accept_len, bonus);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -27,7 +27,6 @@ kv_compact_kernel(BatchArgs a, uint16_t *__restrict__ k_cache, uint16_t *__restr
                   const int32_t *__restrict__ accept_len, int32_t *__restrict__ new_len) {
     extern __shared__ uint4 stage[];      // [kCompactChunk][heads][D/8]
     __shared__ int s_src[kCompactChunk], s_dst[kCompactChunk];
-    __shared__ int s_ok;
     const int b = blockIdx.x;
     uint16_t *cache = blockIdx.y == 0 ? k_cache : v_cache;
     const int h0 = blockIdx.z * kHeadsPerCta;
@@ -35,32 +34,30 @@ kv_compact_kernel(BatchArgs a, uint16_t *__restrict__ k_cache, uint16_t *__restr
     const int vec_per_head = a.D / 8;
     const int vec_per_row = heads * vec_per_head;
 
+    // validation, spread over the block: request descriptors, accept length,
+    // a strictly increasing path from the root, and every page the move touches
     Request r;
-    if (threadIdx.x == 0) {
-        int ok = load_request(a, b, r) ? 1 : 0;
-        int acc = ok ? accept_len[b] : 0;
-        if (ok && (acc < 0 || acc >= r.n || acc + 1 > max_path)) {
-            flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
-            ok = 0;
-        }
-        const int32_t *row = path + (size_t)b * max_path;
-        if (ok && row[0] != 0) ok = 0;
-        for (int k = 1; ok && k <= acc; ++k)
-            if (row[k] <= row[k - 1] || row[k] >= r.n) ok = 0;
-        if (!ok) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
-        // every page the move touches (slots P .. P+n-1) must be mapped
-        if (ok) {
-            for (int pg = r.P / a.page_size; ok && pg <= (r.P + r.n - 1) / a.page_size; ++pg)
-                if (slot_phys_row(a, b, pg * a.page_size) < 0) ok = 0;
-        }
-        s_ok = ok;
-        if (ok && blockIdx.y == 0 && blockIdx.z == 0) new_len[b] = r.P + acc + 1;
-    }
-    __syncthreads();
-    if (!s_ok) return;
-    load_request(a, b, r);
-    const int acc = accept_len[b];
+    const bool req_ok = load_request(a, b, r);
+    const int acc = req_ok ? accept_len[b] : 0;
+    int bad = !req_ok || acc < 0 || acc >= r.n || acc + 1 > max_path;
     const int32_t *row = path + (size_t)b * max_path;
+    if (!bad) {
+        for (int k = threadIdx.x; k <= acc; k += blockDim.x) {
+            const int pk = row[k];
+            if (k == 0 ? pk != 0 : (pk <= row[k - 1] || pk >= r.n)) bad = 1;
+        }
+        const int pg0 = r.P / a.page_size, pg1 = (r.P + r.n - 1) / a.page_size;
+        for (int pg = pg0 + threadIdx.x; pg <= pg1; pg += blockDim.x) {
+            const int page = a.page_table[(size_t)b * a.max_pages_per_req + pg];
+            if (page < 0 || page >= a.num_pages) bad = 1;
+        }
+    }
+    bad = __syncthreads_or(bad);
+    if (bad) {
+        if (threadIdx.x == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+        return;
+    }
+    if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) new_len[b] = r.P + acc + 1;
 
     for (int k0 = 0; k0 <= acc; k0 += kCompactChunk) {
         const int rows = min(kCompactChunk, acc + 1 - k0);

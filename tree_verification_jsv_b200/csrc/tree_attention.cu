@@ -66,10 +66,9 @@ struct AttnParams {
 template <int D>
 struct AttnSmem {
     static constexpr int kQBytes = kRowsPerCta * D * 2;        // Q tile
-    static constexpr int kPBytes = kRowsPerCta * kKeyTile * 2;  // P tile (32 KB)
     static constexpr int kKVBytes = kKeyTile * D * 2;          // one K (or V) tile
     static constexpr int kStageBytes = 2 * kKVBytes;
-    static constexpr int kTotal = kQBytes + kPBytes + kStages * kStageBytes;
+    static constexpr int kTotal = kQBytes + kStages * kStageBytes;
 };
 
 // Byte offset of 16-byte chunk `c` of row `r` in a K-major SW128 operand
@@ -85,8 +84,8 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     using L = AttnSmem<D>;
     constexpr int kHalves = D / 64;
     extern __shared__ uint8_t dsmem[];
-    __shared__ __align__(8) uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
-    __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full, o_done, q_ready, drain_bar;
+    __shared__ __align__(8) uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
+    __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_done, q_ready, drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ volatile int sm_fail;
@@ -115,8 +114,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;
-    uint8_t *sP = smem + L::kQBytes;
-    uint8_t *sKV = sP + L::kPBytes;
+    uint8_t *sKV = smem + L::kQBytes;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -124,13 +122,13 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&v_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
-            mbar_init(&s_empty[s], 4);
+            mbar_init(&p_full[s], 4);
         }
-        mbar_init(&p_full, 4);
         mbar_init(&o_done, 1);
         mbar_init(&q_ready, 4);
         mbar_init(&drain_bar, 1);
@@ -146,8 +144,10 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
-    const uint32_t tS = tmem;              // S buffers: columns [0,128) and [128,256)
-    const uint32_t tO = tmem + 256;        // O: columns [256, 256 + D)
+    // TMEM: S buffers at columns [0,128) and [128,256); P (bf16 pairs) overwrites
+    // the first 64 columns of its own S buffer; O at columns [256, 256 + D)
+    const uint32_t tS = tmem;
+    const uint32_t tO = tmem + 256;
 
     // logical tile index -> first logical slot
     auto tile_slot0 = [&](int j) -> int {
@@ -156,60 +156,106 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 
     if (warp == 0) {
         // ----------------------------------------------------------- producer
-        if (lane == 0 && ntiles > 0) {
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
+        // The whole warp runs the loop: lanes 0..7 look up the 8 physical pages
+        // of the NEXT tile (independent loads, issued before waiting for a free
+        // stage); lane 0 issues the copies, receiving page numbers by shuffle.
+        if (ntiles > 0) {
+            if (lane == 0) {
+                prefetch_tensormap(&tmK);
+                prefetch_tensormap(&tmV);
+            }
             const int oob = a.num_pages * a.page_size;   // fully out-of-bounds slot coordinate
             const int mapped_pages = (r.P + r.n + a.page_size - 1) / a.page_size;
-            long long issued = 0;
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int j = 0; j < ntiles && !abort_sh; ++j) {
-                if (!mbar_wait(&kv_empty[stage], phase ^ 1, &abort_sh)) {
-                    abort_sh = 1;
-                    flag_error(a.dev_status, JSV_ERR_TIMEOUT);
-                    break;
-                }
-                uint8_t *sK = sKV + stage * L::kStageBytes;
-                uint8_t *sV = sK + L::kKVBytes;
-                const int slot0 = tile_slot0(j);
-                mbar_arrive_expect_tx(&k_full[stage], L::kKVBytes);
-                mbar_arrive_expect_tx(&v_full[stage], L::kKVBytes);
-                for (int pg = 0; pg < kKeyTile / 16; ++pg) {
-                    const int lp = slot0 / 16 + pg;          // logical page
-                    int z = oob;
+            auto lookup = [&](int j) -> int {            // slot coordinate of page `lane` of tile j
+                int z = oob;
+                if (lane < kKeyTile / 16) {
+                    const int lp = tile_slot0(j) / 16 + lane;
                     if (lp < mapped_pages) {
                         const int page = a.page_table[(size_t)b * a.max_pages_per_req + lp];
                         if (page >= 0 && page < a.num_pages) z = page * a.page_size;
                         else flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
                     }
-                    for (int h = 0; h < kHalves; ++h) {
-                        tma_load_3d(sK + h * (kKeyTile * 128) + pg * 2048, &tmK, &k_full[stage], h * 64, g, z);
-                        tma_load_3d(sV + h * (kKeyTile * 128) + pg * 2048, &tmV, &v_full[stage], h * 64, g, z);
+                }
+                return z;
+            };
+            long long issued = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            int z_next = lookup(0);
+            bool last_v_issued = true;
+            for (int j = 0; j < ntiles; ++j) {
+                const int z_cur = z_next;
+                if (j + 1 < ntiles) z_next = lookup(j + 1);
+                // K of a stage frees once S of its previous tile is done, V once PV is
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&k_empty[stage], phase ^ 1, &abort_sh) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) {
+                        abort_sh = 1;
+                        flag_error(a.dev_status, JSV_ERR_TIMEOUT);
+                    }
+                    break;
+                }
+                uint8_t *sK = sKV + stage * L::kStageBytes;
+                uint8_t *sV = sK + L::kKVBytes;
+                if (lane == 0) mbar_arrive_expect_tx(&k_full[stage], L::kKVBytes);
+#pragma unroll
+                for (int pg = 0; pg < kKeyTile / 16; ++pg) {
+                    const int z = __shfl_sync(0xffffffffu, z_cur, pg);
+                    if (lane == 0) {
+#pragma unroll
+                        for (int h = 0; h < kHalves; ++h)
+                            tma_load_3d(sK + h * (kKeyTile * 128) + pg * 2048, &tmK, &k_full[stage], h * 64, g, z);
+                    }
+                }
+                if (lane == 0) ok = mbar_wait(&v_empty[stage], phase ^ 1, &abort_sh) ? 1 : 0;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) {
+                        abort_sh = 1;
+                        flag_error(a.dev_status, JSV_ERR_TIMEOUT);
+                    }
+                    last_v_issued = false;      // K of this stage is in flight, V is not
+                    ++issued;
+                    if (++stage == kStages) { stage = 0; phase ^= 1; }
+                    break;
+                }
+                if (lane == 0) mbar_arrive_expect_tx(&v_full[stage], L::kKVBytes);
+#pragma unroll
+                for (int pg = 0; pg < kKeyTile / 16; ++pg) {
+                    const int z = __shfl_sync(0xffffffffu, z_cur, pg);
+                    if (lane == 0) {
+#pragma unroll
+                        for (int h = 0; h < kHalves; ++h)
+                            tma_load_3d(sV + h * (kKeyTile * 128) + pg * 2048, &tmV, &v_full[stage], h * 64, g, z);
                     }
                 }
                 ++issued;
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
+                if (abort_sh) break;
             }
-            if (abort_sh) {
+            if (lane == 0 && abort_sh) {
                 int zero = 0;
                 const long long back = issued < kStages ? issued : kStages;
-                int s = stage;
+                int s2 = stage;
                 uint32_t ph = phase;
                 for (long long i = 0; i < back; ++i) {
-                    if (s == 0) { s = kStages; ph ^= 1; }
-                    --s;
-                    mbar_wait(&k_full[s], ph, (volatile int *)&zero);
-                    mbar_wait(&v_full[s], ph, (volatile int *)&zero);
+                    if (s2 == 0) { s2 = kStages; ph ^= 1; }
+                    --s2;
+                    mbar_wait(&k_full[s2], ph, (volatile int *)&zero);
+                    if (i > 0 || last_v_issued) mbar_wait(&v_full[s2], ph, (volatile int *)&zero);
                 }
             }
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
+        // Issue order: S_0, S_1, PV_0, S_2, PV_1, ...  S_j reuses the TMEM buffer
+        // of P_{j-2}; PV_{j-2} was issued before it and MMAs run in issue order.
         if (lane == 0 && ntiles > 0) {
             const uint32_t id_s = idesc_bf16_f32(128, kKeyTile, false, false);
             const uint32_t id_o = idesc_bf16_f32(128, D, false, true);
-            const uint32_t aQ = smem_addr(sQ), aP = smem_addr(sP);
+            const uint32_t aQ = smem_addr(sQ);
             bool ok = mbar_wait(&q_ready, 0, &abort_sh);
             int kst = 0;                 // stage of tile j
             uint32_t kph = 0;
@@ -219,8 +265,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 if (j < ntiles) {
                     // S_j = Q K_j^T into buffer j % 2
                     const int sb = j & 1;
-                    ok = mbar_wait(&k_full[kst], kph, &abort_sh) &&
-                         mbar_wait(&s_empty[sb], ((j >> 1) & 1) ^ 1, &abort_sh);
+                    ok = mbar_wait(&k_full[kst], kph, &abort_sh);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t aK = smem_addr(sKV + kst * L::kStageBytes);
@@ -232,25 +277,24 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                                     kk > 0);
                     }
                     mma_commit(&s_full[sb]);
+                    mma_commit(&k_empty[kst]);
                     if (++kst == kStages) { kst = 0; kph ^= 1; }
                 }
                 if (j >= 1) {
-                    // O += P_{j-1} V_{j-1}
-                    const int jj = j - 1;
-                    ok = mbar_wait(&p_full, jj & 1, &abort_sh) && mbar_wait(&v_full[vst], vph, &abort_sh);
+                    // O += P_{j-1} V_{j-1}, P read from TMEM
+                    const int jj = j - 1, pb = jj & 1;
+                    ok = mbar_wait(&p_full[pb], (jj >> 1) & 1, &abort_sh) && mbar_wait(&v_full[vst], vph, &abort_sh);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t aV = smem_addr(sKV + vst * L::kStageBytes + L::kKVBytes);
 #pragma unroll
                     for (int kk = 0; kk < kKeyTile / 16; ++kk) {
-                        const uint32_t offp = (kk >> 2) * (kRowsPerCta * 128) + (kk & 3) * 32;
                         // V is MN-major: 16 keys = 16 lines of 128 B; 64-dim blocks 16 KB apart
-                        mma_bf16_ss(tO, desc_kmajor_sw128(aP + offp),
-                                    desc_mnmajor_sw128(aV + kk * 2048, kKeyTile * 128, 1024), id_o,
-                                    (jj > 0 || kk > 0) ? 1u : 0u);
+                        mma_bf16_ts(tO, tS + pb * 128 + kk * 8, desc_mnmajor_sw128(aV + kk * 2048, kKeyTile * 128, 1024),
+                                    id_o, (jj > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(&o_done);
-                    mma_commit(&kv_empty[vst]);
+                    mma_commit(&v_empty[vst]);
                     if (++vst == kStages) { vst = 0; vph ^= 1; }
                 }
             }
@@ -307,6 +351,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         float m_used = -INFINITY, l = 0.f;
         const float sl2 = prm.scale_log2;
         bool ok = true;
+        int o_seen = 0;                              // PV completions observed
         for (int j = 0; j < ntiles; ++j) {
             const int sb = j & 1;
             if (!mbar_wait(&s_full[sb], (j >> 1) & 1, &abort_sh)) ok = false;
@@ -314,113 +359,145 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             tc_fence_after();
             const int slot0 = tile_slot0(j);
             const bool is_tree = j >= (t_end - t_begin);
-            const bool full_tile = !is_tree && slot0 + kKeyTile <= r.P;
             const uint32_t sbase = tS + sb * 128 + lane_addr;
-            // visibility of key column c of this tile for this row
-            auto visible = [&](int c) -> bool {
-                const int slot = slot0 + c;
-                if (!is_tree) return slot < r.P;
-                const int jn = slot - r.P;
-                return jn >= 0 && jn < r.n && row_valid &&
-                       ((anc[row][(jn >> 5) & (kMaxTreeWords - 1)] >> (jn & 31)) & 1u);
-            };
-            // pass 1: row max of the scaled, masked scores
-            float tmax = -INFINITY;
+            // one visibility word per 32-key chunk: bit x <-> key column c0 + x
+            uint32_t vis[kKeyTile / 32];
 #pragma unroll
-            for (int c0 = 0; c0 < kKeyTile; c0 += 32) {
-                uint32_t rr[32];
-                tmem_ld_32x32b_x32(sbase + c0, rr);
-                tmem_ld_wait();
-#pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    const bool vis = full_tile || visible(c0 + x);
-                    tmax = fmaxf(tmax, vis ? __uint_as_float(rr[x]) * sl2 : -INFINITY);
+            for (int c = 0; c < kKeyTile / 32; ++c) {
+                const int s0 = slot0 + c * 32;
+                if (!is_tree) {
+                    const int cnt = r.P - s0;
+                    vis[c] = cnt >= 32 ? 0xffffffffu : (cnt <= 0 ? 0u : ((1u << cnt) - 1u));
+                } else {
+                    const int j0 = s0 - r.P;             // tree node of column c*32 (may be < 0)
+                    uint32_t wv = 0u;
+                    if (row_valid && j0 > -32 && j0 < 32 * kMaxTreeWords) {
+                        if (j0 < 0) {
+                            wv = anc[row][0] << (-j0);
+                        } else {
+                            const int w = j0 >> 5;
+                            const uint32_t lo = anc[row][w];
+                            const uint32_t hi = (w + 1 < kMaxTreeWords) ? anc[row][w + 1] : 0u;
+                            wv = __funnelshift_r(lo, hi, j0 & 31);
+                        }
+                    }
+                    vis[c] = wv;
                 }
             }
+            // pass 1: row max of the raw scores (the scale is positive).  Chunks with
+            // masked columns get -inf written back into TMEM, so pass 2 needs no mask.
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < kKeyTile / 32; c += 2) {
+                uint32_t ra[32], rb[32];
+                tmem_ld_32x32b_x32(sbase + c * 32, ra);
+                tmem_ld_32x32b_x32(sbase + (c + 1) * 32, rb);
+                tmem_ld_wait();
+                if (__any_sync(0xffffffffu, (vis[c] & vis[c + 1]) != 0xffffffffu)) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) {
+                        ra[x] = ((vis[c] >> x) & 1u) ? ra[x] : 0xff800000u;
+                        rb[x] = ((vis[c + 1] >> x) & 1u) ? rb[x] : 0xff800000u;
+                    }
+                    uint32_t h[16];
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) h[x] = ra[x];
+                    tmem_st_32x32b_x16(sbase + c * 32, h);
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) h[x] = ra[16 + x];
+                    tmem_st_32x32b_x16(sbase + c * 32 + 16, h);
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) h[x] = rb[x];
+                    tmem_st_32x32b_x16(sbase + (c + 1) * 32, h);
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) h[x] = rb[16 + x];
+                    tmem_st_32x32b_x16(sbase + (c + 1) * 32 + 16, h);
+                    tmem_st_wait();
+                }
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    mx[x & 3] = fmaxf(mx[x & 3], __uint_as_float(ra[x]));
+                    mx[x & 3] = fmaxf(mx[x & 3], __uint_as_float(rb[x]));
+                }
+            }
+            const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
             // running max with a rescale threshold
             float m_new = m_used;
             if (tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY)) m_new = tmax;
             const float corr = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);   // 0 when m_used = -inf
-            // pass 2: probabilities, their sum, and the packed bf16 row
-            float psum = 0.f;
-            uint32_t pk[kKeyTile / 2];
-#pragma unroll
-            for (int c0 = 0; c0 < kKeyTile; c0 += 32) {
-                uint32_t rr[32];
-                tmem_ld_32x32b_x32(sbase + c0, rr);
-                tmem_ld_wait();
-#pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                    float p0 = 0.f, p1 = 0.f;
-                    if (m_new != -INFINITY) {
-                        if (full_tile || visible(c0 + x)) p0 = fast_exp2(__uint_as_float(rr[x]) * sl2 - m_new);
-                        if (full_tile || visible(c0 + x + 1)) p1 = fast_exp2(__uint_as_float(rr[x + 1]) * sl2 - m_new);
-                    }
-                    psum += p0 + p1;
-                    pk[(c0 + x) / 2] = pack_bf16x2(p0, p1);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[sb]);
-            l = l * corr + psum;
 
-            // O and the P buffer are free once PV_{j-1} has completed
-            if (j >= 1) {
-                if (!mbar_wait(&o_done, (j - 1) & 1, &abort_sh)) ok = false;
+            // O holds P_0..P_{j-1} V under the old max: rescale it (rarely) once
+            // PV_{j-1} has completed.  o_seen counts the PV completions observed;
+            // they are observed one by one, so the parity wait never aliases.
+            if (__any_sync(0xffffffffu, corr != 1.f) && j >= 1) {
+                while (o_seen <= j - 1) {
+                    if (!mbar_wait(&o_done, o_seen & 1, &abort_sh)) ok = false;
+                    ++o_seen;
+                }
                 if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        uint32_t ov[32];
-                        tmem_ld_32x32b_x32(tO + lane_addr + c0, ov);
-                        tmem_ld_wait();
-                        uint32_t lo[16], hi[16];
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t ov[32];
+                    tmem_ld_32x32b_x32(tO + lane_addr + c0, ov);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int x = 0; x < 16; ++x) {
-                            lo[x] = __float_as_uint(__uint_as_float(ov[x]) * corr);
-                            hi[x] = __float_as_uint(__uint_as_float(ov[16 + x]) * corr);
-                        }
-                        tmem_st_32x32b_x16(tO + lane_addr + c0, lo);
-                        tmem_st_32x32b_x16(tO + lane_addr + c0 + 16, hi);
-                    }
-                    tmem_st_wait();
+                    for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * corr);
+                    tmem_st_32x32b_x32(tO + lane_addr + c0, ov);
                 }
+                tmem_st_wait();
             }
-            m_used = m_new;
-            // P row (bf16) into the K-major SW128 layout: keys 0-63 and 64-127 in two regions
+
+            // pass 2: probabilities (masked columns hold -inf and give 0), their sum,
+            // and the bf16 P row stored into the first 64 columns of this S buffer
+            const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < kKeyTile / 8; ++c) {
-                const uint4 v = make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
-                *reinterpret_cast<uint4 *>(sP + (c >> 3) * (kRowsPerCta * 128) + sw128_offset(row, c & 7)) = v;
+            for (int c = 0; c < kKeyTile / 32; c += 2) {
+                uint32_t ra[32], rb[32];
+                tmem_ld_32x32b_x32(sbase + c * 32, ra);
+                tmem_ld_32x32b_x32(sbase + (c + 1) * 32, rb);
+                tmem_ld_wait();
+                uint32_t pk[32];
+#pragma unroll
+                for (int x = 0; x < 32; x += 2) {
+                    const float a0 = fast_exp2(fmaf(__uint_as_float(ra[x]), sl2, neg_m));
+                    const float a1 = fast_exp2(fmaf(__uint_as_float(ra[x + 1]), sl2, neg_m));
+                    const float b0 = fast_exp2(fmaf(__uint_as_float(rb[x]), sl2, neg_m));
+                    const float b1 = fast_exp2(fmaf(__uint_as_float(rb[x + 1]), sl2, neg_m));
+                    ps[(x >> 1) & 3] += (a0 + a1) + (b0 + b1);
+                    pk[x / 2] = pack_bf16x2(a0, a1);
+                    pk[16 + x / 2] = pack_bf16x2(b0, b1);
+                }
+                // keys [32c, 32c + 64) -> packed columns [16c, 16c + 32): columns the
+                // loads above have already consumed
+                tmem_st_32x32b_x32(sbase + c * 16, pk);
             }
-            fence_async_smem();
+            const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            l = l * corr + psum;
+            m_used = m_new;
+            tmem_st_wait();
+            // observe PV_{j-1} before handing over P_j (PV_j cannot start before that)
+            while (o_seen <= j - 1) {
+                if (!mbar_wait(&o_done, o_seen & 1, &abort_sh)) ok = false;
+                ++o_seen;
+            }
+            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full);
+            if (lane == 0) mbar_arrive(&p_full[sb]);
         }
 
         // final partial: O (unnormalised), running max (log2 domain) and sum
-        float ofin[D];
         bool have_o = ok && ntiles > 0;
         if (have_o) {
-            if (!mbar_wait(&o_done, (ntiles - 1) & 1, &abort_sh)) ok = false;
+            while (o_seen <= ntiles - 1) {
+                if (!mbar_wait(&o_done, o_seen & 1, &abort_sh)) ok = false;
+                ++o_seen;
+            }
             if (__any_sync(0xffffffffu, !ok)) have_o = false;
         }
-        if (have_o) {
-            tc_fence_after();
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t rr[32];
-                tmem_ld_32x32b_x32(tO + lane_addr + c0, rr);
-                tmem_ld_wait();
-#pragma unroll
-                for (int x = 0; x < 32; ++x) ofin[c0 + x] = __uint_as_float(rr[x]);
-            }
-        } else {
-#pragma unroll
-            for (int x = 0; x < D; ++x) ofin[x] = 0.f;
+        if (!have_o) {
             m_used = -INFINITY;
             l = 0.f;
             if (!ok) {
@@ -428,12 +505,28 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 flag_error(a.dev_status, JSV_ERR_TIMEOUT);
             }
         }
-        if (row_valid) {
-            const size_t rows = (size_t)a.total_nodes * a.Hq;
-            const size_t row_id = (size_t)(r.base + node) * a.Hq + head;
-            float4 *po = reinterpret_cast<float4 *>(prm.ws_o + ((size_t)split * rows + row_id) * D);
+        const size_t rows = (size_t)a.total_nodes * a.Hq;
+        const size_t row_id = (size_t)(r.base + min(node, r.n - 1)) * a.Hq + head;
+        float4 *po = reinterpret_cast<float4 *>(prm.ws_o + ((size_t)split * rows + row_id) * D);
+        if (have_o) tc_fence_after();
 #pragma unroll
-            for (int x = 0; x < D / 4; ++x) po[x] = make_float4(ofin[4 * x], ofin[4 * x + 1], ofin[4 * x + 2], ofin[4 * x + 3]);
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t rr[32];
+            if (have_o) {
+                tmem_ld_32x32b_x32(tO + lane_addr + c0, rr);     // warp-collective: all lanes
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int x = 0; x < 32; ++x) rr[x] = 0u;
+            }
+            if (row_valid) {
+#pragma unroll
+                for (int x = 0; x < 8; ++x)
+                    po[c0 / 4 + x] = make_float4(__uint_as_float(rr[4 * x]), __uint_as_float(rr[4 * x + 1]),
+                                                 __uint_as_float(rr[4 * x + 2]), __uint_as_float(rr[4 * x + 3]));
+            }
+        }
+        if (row_valid) {
             prm.ws_ml[((size_t)split * rows + row_id) * 2 + 0] = m_used;
             prm.ws_ml[((size_t)split * rows + row_id) * 2 + 1] = l;
         }
