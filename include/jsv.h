@@ -206,6 +206,14 @@ JSV_API jsv_status jsv_lmhead_argmax_noalloc(const uint16_t *hidden, const uint1
  * launches inside a timed region; not tied to any stream order. */
 JSV_API uint64_t jsv_kernel_launches(void);
 
+/* Text of the last CUDA error behind a JSV_ERR_CUDA returned to the calling
+ * host thread (a launch or runtime call that failed), or a fixed message if
+ * none was recorded; for a failed kernel launch it also names the kernel's
+ * registers and shared memory against the launch.  The string belongs to the
+ * calling thread and stays valid until its next call; later successful calls
+ * do not clear it. */
+JSV_API const char *jsv_last_error_string(void);
+
 /* Static string for a status code. */
 JSV_API const char *jsv_status_string(jsv_status status);
 

@@ -3,10 +3,20 @@
 #include "jsv_internal.cuh"
 
 #include <atomic>
+#include <cstdio>
 
 namespace jsv {
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+static thread_local char t_launch_note[256] = {0};
+void note_launch_failure(const char *what, int regs, int max_threads, size_t static_smem, int max_dyn_smem,
+                         int threads, size_t dyn_smem) {
+    snprintf(t_launch_note, sizeof t_launch_note,
+             "%s launch: %d regs/thread, max %d threads/block, %zu B static + %zu B dynamic smem "
+             "requested (limit %d B dynamic), %d threads",
+             what, regs, max_threads, static_smem, dyn_smem, max_dyn_smem, threads);
+}
 }  // namespace jsv
 
 namespace {
@@ -27,7 +37,13 @@ jsv_status check_batch(const jsv_batch *b) {
     return JSV_OK;
 }
 
-jsv_status from_cuda(cudaError_t e) { return e == cudaSuccess ? JSV_OK : JSV_ERR_CUDA; }
+thread_local cudaError_t t_last_error = cudaSuccess;
+
+jsv_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return JSV_OK;
+    t_last_error = e;
+    return JSV_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -107,6 +123,14 @@ const char *jsv_status_string(jsv_status status) {
 }
 
 int32_t jsv_version(void) { return 100; }
+
+const char *jsv_last_error_string(void) {
+    static thread_local char buf[512];
+    if (t_last_error == cudaSuccess) return "no CUDA error recorded";
+    snprintf(buf, sizeof buf, "%s%s%s", cudaGetErrorString(t_last_error), jsv::t_launch_note[0] ? " -- " : "",
+             jsv::t_launch_note);
+    return buf;
+}
 
 uint64_t jsv_kernel_launches(void) { return jsv::g_launches.load(std::memory_order_relaxed); }
 

@@ -70,6 +70,11 @@ __device__ __forceinline__ long long slot_phys_row(const BatchArgs &a, int b, in
 // Count of kernel launches issued by the library (see jsv_kernel_launches).
 void count_launches(int n);
 
+// Record the resources of a kernel whose launch failed, for
+// jsv_last_error_string (thread-local).
+void note_launch_failure(const char *what, int regs, int max_threads, size_t static_smem, int max_dyn_smem,
+                         int threads, size_t dyn_smem);
+
 }  // namespace jsv
 
 // Launchers (defined in the kernel files, called from jsv_api.cu).

@@ -5,28 +5,35 @@
 // prefix slots [0, P) and to slot P + j for every ancestor-or-self j of i.
 //
 // Work decomposition (one CTA per unit):
-//   (request b, KV head g, M-tile of 128 query rows, KV split s)
+//   (request b, KV head g, tile of 256 query rows, KV split s)
 // Query rows of (b, g) pack the G = Hq/Hkv heads that share KV head g:
 // row r <-> node r / G, head g*G + r % G, so every K/V tile loaded serves
-// G*128/G = 128 query rows (GQA packing).  The prefix is cut into 128-key
-// tiles that start on page boundaries; split s takes a contiguous run of
-// them, and the last split also takes the tree tiles, which cover slots
-// [P & ~15, P + N) and apply the ancestor mask.  Each split writes an
-// unnormalised fp32 partial (O, row max, row sum); a small combine kernel
-// merges the splits with log-sum-exp rescaling and rounds to bf16.
+// 256 query rows (GQA packing).  The 256 rows form two 128-row groups that
+// take turns on the tensor core.  The prefix is cut into 128-key tiles that
+// start on page boundaries; split s takes a contiguous run of them, and the
+// last split also takes the tree tiles, which cover slots [P & ~15, P + N)
+// and apply the ancestor mask.  Each split writes an unnormalised fp32
+// partial (O, row max, row sum); a small combine kernel merges the splits
+// with log-sum-exp rescaling and rounds to bf16.
 //
-// Per CTA, 6 warps:
+// Per CTA, 10 warps:
 //   warp 0      TMA producer: K and V of each 128-key tile, one 16-slot
-//               page x 64-dim box per copy, into a 2-stage ring
-//   warp 1      TMEM allocator and single-thread MMA issuer:
-//               S_j = Q K_j^T into one of two TMEM S buffers, then
-//               O += P_{j-1} V_{j-1} once softmax has written P_{j-1}
-//   warps 2..5  softmax: one query row per thread; load S_j from TMEM,
-//               mask, online softmax in the log2 domain, write P_j (bf16)
-//               to shared memory; rescale O in TMEM only when the running
-//               max grows by more than 8 (2^8), which keeps exp2 arguments
-//               bounded without touching O on most tiles
-// Shared memory: Q (16 KB per 64 dims), P (32 KB), 2 x (K, V) stages.
+//               page x 64-dim box per copy, into a 2-stage ring; the warp
+//               looks up the next tile's pages while it waits for a stage
+//   warp 1      TMEM allocator and single-thread MMA issuer, in the order
+//               S0_0 S1_0 | PV0_0 S0_1 PV1_0 S1_1 | PV0_1 S0_2 ...
+//               (Sg_j = Q_g K_j^T, PVg_j: O_g += P_g V_j with P read from TMEM)
+//   warps 2..5  softmax of row group 0, warps 6..9 of row group 1: one query
+//               row per thread; masked online softmax in the log2 domain;
+//               P_j (bf16) is written over its own S buffer in TMEM; O is
+//               rescaled in TMEM only when the running max grows by more
+//               than 8 (2^8), which keeps exp2 arguments bounded
+// While one group computes its softmax the tensor core runs the other
+// group's products, so neither the exp2 pipe nor the tensor pipe waits on
+// the other for long.
+// TMEM columns: S/P of group 0 [0,128), of group 1 [128,256); O of group 0
+// [256, 256+D), of group 1 [256+D, 256+2D).
+// Shared memory: Q (2 groups x 16 KB per 64 dims), 2 x (K, V) stages.
 #include "jsv_internal.cuh"
 #include "sm100.cuh"
 
@@ -36,9 +43,11 @@ namespace jsv {
 
 using namespace sm100;
 
-constexpr int kAttnThreads = 192;
+constexpr int kGroups = 2;
+constexpr int kGroupRows = 128;
+constexpr int kRowsPerCta = kGroups * kGroupRows;
+constexpr int kAttnThreads = 64 + kGroups * 128;
 constexpr int kKeyTile = 128;
-constexpr int kRowsPerCta = 128;
 constexpr int kStages = 2;
 constexpr int kMaxTreeWords = 16;          // 512 nodes
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -65,7 +74,8 @@ struct AttnParams {
 
 template <int D>
 struct AttnSmem {
-    static constexpr int kQBytes = kRowsPerCta * D * 2;        // Q tile
+    static constexpr int kQGroupBytes = kGroupRows * D * 2;    // one row group's Q
+    static constexpr int kQBytes = kGroups * kQGroupBytes;
     static constexpr int kKVBytes = kKeyTile * D * 2;          // one K (or V) tile
     static constexpr int kStageBytes = 2 * kKVBytes;
     static constexpr int kTotal = kQBytes + kStages * kStageBytes;
@@ -85,7 +95,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     constexpr int kHalves = D / 64;
     extern __shared__ uint8_t dsmem[];
     __shared__ __align__(8) uint64_t k_full[kStages], v_full[kStages], k_empty[kStages], v_empty[kStages];
-    __shared__ __align__(8) uint64_t s_full[2], p_full[2], o_done, q_ready, drain_bar;
+    __shared__ __align__(8) uint64_t s_full[kGroups], p_full[kGroups], o_done[kGroups], q_ready, drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ volatile int sm_fail;
@@ -103,6 +113,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     const int rows_total = r.n * G;
     if (m0 >= rows_total) return;
     const int rows_here = min(kRowsPerCta, rows_total - m0);
+    const int ngroups = rows_here > kGroupRows ? 2 : 1;     // a group with no rows is skipped
 
     // tile schedule for this split
     const int prefix_tiles = (r.P + kKeyTile - 1) / kKeyTile;
@@ -125,12 +136,12 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             mbar_init(&k_empty[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kGroups; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], 4);
+            mbar_init(&o_done[s], 1);
         }
-        mbar_init(&o_done, 1);
-        mbar_init(&q_ready, 4);
+        mbar_init(&q_ready, 4 * kGroups);
         mbar_init(&drain_bar, 1);
         abort_sh = 0;
         sm_fail = 0;
@@ -144,10 +155,6 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
-    // TMEM: S buffers at columns [0,128) and [128,256); P (bf16 pairs) overwrites
-    // the first 64 columns of its own S buffer; O at columns [256, 256 + D)
-    const uint32_t tS = tmem;
-    const uint32_t tO = tmem + 256;
 
     // logical tile index -> first logical slot
     auto tile_slot0 = [&](int j) -> int {
@@ -186,7 +193,8 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             for (int j = 0; j < ntiles; ++j) {
                 const int z_cur = z_next;
                 if (j + 1 < ntiles) z_next = lookup(j + 1);
-                // K of a stage frees once S of its previous tile is done, V once PV is
+                // K of a stage frees once both groups' S of its previous tile are
+                // done, V once both groups' PV are
                 int ok = 1;
                 if (lane == 0) ok = mbar_wait(&k_empty[stage], phase ^ 1, &abort_sh) ? 1 : 0;
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -250,52 +258,65 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
-        // Issue order: S_0, S_1, PV_0, S_2, PV_1, ...  S_j reuses the TMEM buffer
-        // of P_{j-2}; PV_{j-2} was issued before it and MMAs run in issue order.
+        // S of a group reuses the TMEM of that group's previous P; the PV that
+        // reads it was issued earlier and MMAs run in issue order.
         if (lane == 0 && ntiles > 0) {
             const uint32_t id_s = idesc_bf16_f32(128, kKeyTile, false, false);
             const uint32_t id_o = idesc_bf16_f32(128, D, false, true);
             const uint32_t aQ = smem_addr(sQ);
             bool ok = mbar_wait(&q_ready, 0, &abort_sh);
-            int kst = 0;                 // stage of tile j
-            uint32_t kph = 0;
-            int vst = 0;                 // stage of tile j-1 (for PV)
-            uint32_t vph = 0;
-            for (int j = 0; ok && j <= ntiles; ++j) {
-                if (j < ntiles) {
-                    // S_j = Q K_j^T into buffer j % 2
-                    const int sb = j & 1;
-                    ok = mbar_wait(&k_full[kst], kph, &abort_sh);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t aK = smem_addr(sKV + kst * L::kStageBytes);
+            auto issue_s = [&](int grp, int kstage) {
+                const uint32_t aK = smem_addr(sKV + kstage * L::kStageBytes);
+                const uint32_t aQg = aQ + grp * L::kQGroupBytes;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * (kRowsPerCta * 128) + (kk & 3) * 32;
-                        const uint32_t offk = (kk >> 2) * (kKeyTile * 128) + (kk & 3) * 32;
-                        mma_bf16_ss(tS + sb * 128, desc_kmajor_sw128(aQ + off), desc_kmajor_sw128(aK + offk), id_s,
-                                    kk > 0);
-                    }
-                    mma_commit(&s_full[sb]);
-                    mma_commit(&k_empty[kst]);
-                    if (++kst == kStages) { kst = 0; kph ^= 1; }
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kGroupRows * 128) + (kk & 3) * 32;
+                    const uint32_t offk = (kk >> 2) * (kKeyTile * 128) + (kk & 3) * 32;
+                    mma_bf16_ss(tmem + grp * 128, desc_kmajor_sw128(aQg + off), desc_kmajor_sw128(aK + offk),
+                                id_s, kk > 0);
                 }
-                if (j >= 1) {
-                    // O += P_{j-1} V_{j-1}, P read from TMEM
-                    const int jj = j - 1, pb = jj & 1;
-                    ok = mbar_wait(&p_full[pb], (jj >> 1) & 1, &abort_sh) && mbar_wait(&v_full[vst], vph, &abort_sh);
+                mma_commit(&s_full[grp]);
+            };
+            auto issue_pv = [&](int grp, int vstage, int jj) {
+                const uint32_t aV = smem_addr(sKV + vstage * L::kStageBytes + L::kKVBytes);
+#pragma unroll
+                for (int kk = 0; kk < kKeyTile / 16; ++kk) {
+                    // V is MN-major: 16 keys = 16 lines of 128 B; 64-dim blocks 16 KB apart
+                    mma_bf16_ts(tmem + 256 + grp * D, tmem + grp * 128 + kk * 8,
+                                desc_mnmajor_sw128(aV + kk * 2048, kKeyTile * 128, 1024), id_o,
+                                (jj > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&o_done[grp]);
+            };
+            // prologue: S of tile 0 for both groups
+            if (ok) ok = mbar_wait(&k_full[0], 0, &abort_sh);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                if (ngroups > 1) issue_s(1, 0);
+                mma_commit(&k_empty[0]);
+            }
+            for (int j = 0; ok && j < ntiles; ++j) {
+                const int st = j % kStages;
+                const uint32_t ph = (uint32_t)((j / kStages) & 1);
+                const int stn = (j + 1) % kStages;
+                const uint32_t phn = (uint32_t)(((j + 1) / kStages) & 1);
+                const bool more = j + 1 < ntiles;
+                for (int grp = 0; grp < ngroups; ++grp) {
+                    ok = mbar_wait(&p_full[grp], j & 1, &abort_sh) && (grp > 0 || mbar_wait(&v_full[st], ph, &abort_sh));
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t aV = smem_addr(sKV + vst * L::kStageBytes + L::kKVBytes);
-#pragma unroll
-                    for (int kk = 0; kk < kKeyTile / 16; ++kk) {
-                        // V is MN-major: 16 keys = 16 lines of 128 B; 64-dim blocks 16 KB apart
-                        mma_bf16_ts(tO, tS + pb * 128 + kk * 8, desc_mnmajor_sw128(aV + kk * 2048, kKeyTile * 128, 1024),
-                                    id_o, (jj > 0 || kk > 0) ? 1u : 0u);
+                    issue_pv(grp, st, j);
+                    if (grp == ngroups - 1) mma_commit(&v_empty[st]);
+                    if (more) {
+                        if (grp == 0) {
+                            ok = mbar_wait(&k_full[stn], phn, &abort_sh);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                        issue_s(grp, stn);
+                        if (grp == ngroups - 1) mma_commit(&k_empty[stn]);
                     }
-                    mma_commit(&o_done);
-                    mma_commit(&v_empty[vst]);
-                    if (++vst == kStages) { vst = 0; vph ^= 1; }
                 }
             }
             if (!ok) {
@@ -308,17 +329,21 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         }
     } else {
         // ----------------------------------------------------------- softmax
-        const int sub = warp & 3;
-        const int row = sub * 32 + lane;            // TMEM lane == query row in the tile
+        const int grp = (warp - 2) >> 2;             // row group of this warp
+        const int sub = warp & 3;                    // TMEM lanes this warp may access
+        const int grow = sub * 32 + lane;            // row within the group == TMEM lane
+        const int row = grp * kGroupRows + grow;     // row within the CTA tile
         const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
-        const int et = threadIdx.x - 64;             // 0..127
+        const uint32_t tS = tmem + grp * 128;
+        const uint32_t tO = tmem + 256 + grp * D;
+        const int et = threadIdx.x - 64;             // 0..255
         const bool row_valid = row < rows_here;
         const int rg = m0 + row;                     // row within (b, g)
         const int node = rg / G;                     // request-local node
         const int head = g * G + rg % G;
 
-        // Q tile: rows x D bf16 into the K-major SW128 layout (zero rows past the end)
-        for (int e = et; e < kRowsPerCta * (D / 8); e += 128) {
+        // Q of both groups: rows x D bf16 in the K-major SW128 layout (zero rows past the end)
+        for (int e = et; e < kRowsPerCta * (D / 8); e += kGroups * 128) {
             const int rr = e / (D / 8), c = e % (D / 8);
             uint4 v = make_uint4(0, 0, 0, 0);
             if (rr < rows_here) {
@@ -326,7 +351,8 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 const uint16_t *src = prm.q + ((size_t)(r.base + rgg / G) * a.Hq + g * G + rgg % G) * D + c * 8;
                 v = *reinterpret_cast<const uint4 *>(src);
             }
-            *reinterpret_cast<uint4 *>(sQ + (c >> 3) * (kRowsPerCta * 128) + sw128_offset(rr, c & 7)) = v;
+            *reinterpret_cast<uint4 *>(sQ + (rr / kGroupRows) * L::kQGroupBytes + (c >> 3) * (kGroupRows * 128) +
+                                       sw128_offset(rr % kGroupRows, c & 7)) = v;
         }
         // ancestor-or-self bitsets of this tile's rows (only the last split uses them)
         if (tree_tiles > 0 && row_valid) {
@@ -341,7 +367,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             }
         }
         fence_async_smem();
-        named_barrier(1, 128);
+        named_barrier(1, kGroups * 128);
         if (sm_fail) {
             if (et == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
         }
@@ -352,14 +378,14 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         const float sl2 = prm.scale_log2;
         bool ok = true;
         int o_seen = 0;                              // PV completions observed
-        for (int j = 0; j < ntiles; ++j) {
-            const int sb = j & 1;
-            if (!mbar_wait(&s_full[sb], (j >> 1) & 1, &abort_sh)) ok = false;
+        const int my_tiles = grp < ngroups ? ntiles : 0;
+        for (int j = 0; j < my_tiles; ++j) {
+            if (!mbar_wait(&s_full[grp], j & 1, &abort_sh)) ok = false;
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             tc_fence_after();
             const int slot0 = tile_slot0(j);
             const bool is_tree = j >= (t_end - t_begin);
-            const uint32_t sbase = tS + sb * 128 + lane_addr;
+            const uint32_t sbase = tS + lane_addr;
             // one visibility word per 32-key chunk: bit x <-> key column c0 + x
             uint32_t vis[kKeyTile / 32];
 #pragma unroll
@@ -431,7 +457,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             // they are observed one by one, so the parity wait never aliases.
             if (__any_sync(0xffffffffu, corr != 1.f) && j >= 1) {
                 while (o_seen <= j - 1) {
-                    if (!mbar_wait(&o_done, o_seen & 1, &abort_sh)) ok = false;
+                    if (!mbar_wait(&o_done[grp], o_seen & 1, &abort_sh)) ok = false;
                     ++o_seen;
                 }
                 if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
@@ -479,20 +505,20 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             tmem_st_wait();
             // observe PV_{j-1} before handing over P_j (PV_j cannot start before that)
             while (o_seen <= j - 1) {
-                if (!mbar_wait(&o_done, o_seen & 1, &abort_sh)) ok = false;
+                if (!mbar_wait(&o_done[grp], o_seen & 1, &abort_sh)) ok = false;
                 ++o_seen;
             }
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[sb]);
+            if (lane == 0) mbar_arrive(&p_full[grp]);
         }
 
         // final partial: O (unnormalised), running max (log2 domain) and sum
-        bool have_o = ok && ntiles > 0;
+        bool have_o = ok && my_tiles > 0;
         if (have_o) {
-            while (o_seen <= ntiles - 1) {
-                if (!mbar_wait(&o_done, o_seen & 1, &abort_sh)) ok = false;
+            while (o_seen <= my_tiles - 1) {
+                if (!mbar_wait(&o_done[grp], o_seen & 1, &abort_sh)) ok = false;
                 ++o_seen;
             }
             if (__any_sync(0xffffffffu, !ok)) have_o = false;
@@ -650,6 +676,14 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
     }
     dim3 grid((a.max_nodes * G + kRowsPerCta - 1) / kRowsPerCta, S, a.B * a.Hkv);
     tree_attention_tc_kernel<D><<<grid, kAttnThreads, smem, st>>>(tmK, tmV, prm);
+    cudaError_t le = cudaGetLastError();
+    if (le != cudaSuccess) {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, tree_attention_tc_kernel<D>) == cudaSuccess)
+            note_launch_failure("tree attention", fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes,
+                                fa.maxDynamicSharedSizeBytes, kAttnThreads, smem);
+        return le;
+    }
     dim3 cgrid((a.max_nodes * G + kCombineWarps - 1) / kCombineWarps, 1, a.B * a.Hkv);
     tree_attention_combine_kernel<D><<<cgrid, kCombineWarps * 32, 0, st>>>(a, S, prm.ws_o, prm.ws_ml, out);
     count_launches(2);

@@ -23,7 +23,7 @@ JSV_ERR_DEVICE_INPUT = 5
 EXPORTS = ("jsv_tree_attention_workspace_size", "jsv_tree_attention",
            "jsv_lmhead_argmax_workspace_size", "jsv_lmhead_argmax", "jsv_accept_path",
            "jsv_kv_compact", "jsv_status_string", "jsv_version", "jsv_kernel_launches",
-           "jsv_lmhead_argmax_noalloc")
+           "jsv_lmhead_argmax_noalloc", "jsv_last_error_string")
 
 # Largest node count jsv_lmhead_argmax_noalloc accepts (JSV_NOALLOC_MAX_NODES).
 NOALLOC_MAX_NODES = 8192
@@ -31,7 +31,10 @@ NOALLOC_MAX_NODES = 8192
 
 class JsvError(RuntimeError):
     def __init__(self, fn: str, status: int):
-        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+        msg = f"{fn}: {status_string(status)} (status {status})"
+        if status == JSV_ERR_CUDA:
+            msg += f": {load().jsv_last_error_string().decode()}"
+        super().__init__(msg)
         self.status = status
 
 
@@ -78,6 +81,8 @@ def load() -> ctypes.CDLL:
     lib.jsv_version.restype = i32
     lib.jsv_lmhead_argmax_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
     lib.jsv_lmhead_argmax_noalloc.restype = ctypes.c_int
+    lib.jsv_last_error_string.argtypes = []
+    lib.jsv_last_error_string.restype = ctypes.c_char_p
     lib.jsv_kernel_launches.argtypes = []
     lib.jsv_kernel_launches.restype = ctypes.c_uint64
     _lib = lib
