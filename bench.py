@@ -5,8 +5,9 @@ A step is one pass of the whole hot path over one batch of synthetic input:
 tree attention, LM head + argmax, accept walk and KV compaction, i.e. the
 four calls of ``include/jsv.h`` on one stream.  Inputs are resident in HBM
 when the timed region starts; L2 is flushed (a 512 MB write) before every
-timed step, outside its events.  Step and per-call times come from CUDA
-events on the launching stream.
+timed step, outside its events.  The headline times whole steps with CUDA
+events on the launching stream; a second timed pass of the same steps puts
+an event between the calls for the per-call durations (the roofline).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
   python bench.py --impl reference ...   # the CPU oracle on the host cores
@@ -292,7 +293,8 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    # timed region 1 (the headline): whole steps, events only around each step
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -300,22 +302,34 @@ def run_gpu(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clocks:
         for i in range(K):
             flush.fill_(i & 0xFF)
-            e = ev[i]
-            e[0].record(stream)
-            st.attention()
-            e[1].record(stream)
-            st.lmhead()
-            e[2].record(stream)
-            st.accept()
-            e[3].record(stream)
-            st.compact()
-            e[4].record(stream)
+            ev[i][0].record(stream)
+            st.run()
+            ev[i][1].record(stream)
         torch.cuda.synchronize()
     launches = jsv.jsv_kernel_launches() - launches0
     if world > 1:
         torch.distributed.barrier()
-    per = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)] for i in range(K)])
-    step_ms = float(per.sum(axis=1).mean())
+    step_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    assert int(st.status.item()) == 0
+
+    # timed region 2: the same steps with an event between calls, for the
+    # per-call durations (the dominant kernel's roofline uses these)
+    evc = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        e = evc[i]
+        e[0].record(stream)
+        st.attention()
+        e[1].record(stream)
+        st.lmhead()
+        e[2].record(stream)
+        st.accept()
+        e[3].record(stream)
+        st.compact()
+        e[4].record(stream)
+    torch.cuda.synchronize()
+    per = np.array([[evc[i][j].elapsed_time(evc[i][j + 1]) for j in range(4)] for i in range(K)])
     call_ms = per.mean(axis=0)
     assert int(st.status.item()) == 0
 
@@ -382,6 +396,7 @@ def run_gpu(args, rank, world, local_rank):
         "north_star_bytes": model["north_star_bytes"],
         "call_us": {n: float(call_ms[j] * 1e3) for j, n in enumerate(names)},
         "call_share": share,
+        "call_sum_us": float(call_ms.sum() * 1e3),
         "roofline": roof,
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),

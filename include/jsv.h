@@ -120,7 +120,8 @@ JSV_API jsv_status jsv_tree_attention(const jsv_batch *batch, const uint16_t *q,
                               float scale, uint16_t *out,
                               void *workspace, size_t workspace_bytes, void *stream);
 
-/* Bytes of scratch jsv_lmhead_argmax needs (one 64-bit key per node). */
+/* Bytes of scratch jsv_lmhead_argmax needs (one 64-bit key per node and a
+ * completion counter). */
 JSV_API size_t jsv_lmhead_argmax_workspace_size(int32_t T, int32_t d, int32_t V);
 
 /*
@@ -184,8 +185,8 @@ JSV_API jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uin
  * workspace argument.  The caller still passes inputs and outputs.
  *   - T must be <= JSV_NOALLOC_MAX_NODES, else JSV_ERR_UNSUPPORTED; the
  *     other arguments follow jsv_lmhead_argmax.
- *   - The array (JSV_NOALLOC_MAX_NODES * 8 bytes) is held on every GPU that
- *     loads the library until the process exits.
+ *   - The array ((JSV_NOALLOC_MAX_NODES + 1) * 8 bytes) is held on every GPU
+ *     that loads the library until the process exits.
  *   - The first call on a device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
  *     stream capture.

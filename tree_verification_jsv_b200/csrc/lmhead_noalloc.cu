@@ -9,7 +9,7 @@
 // entry point whose scratch -- one 64-bit argmax key per node -- lives in a
 // fixed file-scope device array instead of a workspace argument.
 //
-// The array is JSV_NOALLOC_MAX_NODES keys (64 KiB).  Every GPU that loads
+// The array is JSV_NOALLOC_MAX_NODES keys plus one counter word (64 KiB + 8 B).  Every GPU that loads
 // the library holds it until the process exits.  Host code must not pass
 // the array's name to a kernel (on the host it is only a stand-in for the
 // symbol); its device address is looked up once per device, with that
@@ -20,7 +20,8 @@
 
 namespace jsv {
 
-static __device__ __align__(256) unsigned long long g_lmhead_noalloc_keys[JSV_NOALLOC_MAX_NODES];
+// one 64-bit argmax key per node plus the LM-head kernel's completion counter
+static __device__ __align__(256) unsigned long long g_lmhead_noalloc_keys[JSV_NOALLOC_MAX_NODES + 1];
 
 namespace {
 std::mutex g_noalloc_mu;
@@ -58,7 +59,9 @@ jsv_status jsv_lmhead_argmax_noalloc(const uint16_t *hidden, const uint16_t *w, 
         return JSV_ERR_INVALID_ARG;
     void *scratch = nullptr;
     if (jsv::noalloc_scratch(&scratch) != cudaSuccess) return JSV_ERR_CUDA;
-    // the launcher clears the keys it uses before the kernel runs
+    // the launcher clears the keys and counter it uses before the kernel runs
+    static_assert(sizeof(jsv::g_lmhead_noalloc_keys) >= (JSV_NOALLOC_MAX_NODES + 1) * sizeof(unsigned long long),
+                  "scratch must hold the keys and the completion counter");
     cudaError_t e = jsv::launch_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, scratch,
                                               static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? JSV_OK : JSV_ERR_CUDA;
