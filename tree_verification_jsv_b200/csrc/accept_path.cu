@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(kWalkWarps * 32)
 accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
                    const int32_t *__restrict__ argmax, int max_path, int32_t *__restrict__ path,
                    int32_t *__restrict__ accept_len, int32_t *__restrict__ bonus) {
+    pdl_allow_dependents();
+    pdl_wait_predecessor();
     // the request's parent / token / target-choice arrays, staged once
     __shared__ int32_t s_par[kWalkWarps][kWalkMaxNodes];
     __shared__ int32_t s_tok[kWalkWarps][kWalkMaxNodes];
@@ -82,9 +84,10 @@ cudaError_t launch_accept_path(const BatchArgs &a, const int32_t *tokens, const 
                                int max_path, int32_t *path, int32_t *accept_len, int32_t *bonus,
                                cudaStream_t st) {
     dim3 grid((a.B + kWalkWarps - 1) / kWalkWarps);
-    accept_path_kernel<<<grid, kWalkWarps * 32, 0, st>>>(a, tokens, argmax, max_path, path, accept_len, bonus);
+    cudaError_t e = launch_pdl(accept_path_kernel, grid, dim3(kWalkWarps * 32), 0, st, a, tokens, argmax, max_path,
+                               path, accept_len, bonus);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace jsv

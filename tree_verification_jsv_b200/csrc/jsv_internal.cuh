@@ -26,6 +26,19 @@ inline BatchArgs to_args(const jsv_batch *b) {
     return a;
 }
 
+// Programmatic dependent launch: every kernel of the library is launched so
+// that the next kernel in the stream may be scheduled before it finishes.
+// A kernel lets its dependents be scheduled at entry (they can only start
+// once every CTA of this grid has started or exited, so they never take SMs
+// this grid still needs), and waits for its own predecessor to complete --
+// and its memory to be visible -- before it reads any input.
+__device__ __forceinline__ void pdl_allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_predecessor() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void flag_error(int32_t *status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
@@ -74,6 +87,23 @@ void count_launches(int n);
 // jsv_last_error_string (thread-local).
 void note_launch_failure(const char *what, int regs, int max_threads, size_t static_smem, int max_dyn_smem,
                          int threads, size_t dyn_smem);
+
+// Launch `kernel` on `st` with programmatic stream serialization allowed.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 }  // namespace jsv
 

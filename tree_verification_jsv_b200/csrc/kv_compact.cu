@@ -25,6 +25,8 @@ __global__ void __launch_bounds__(kCompactThreads)
 kv_compact_kernel(BatchArgs a, uint16_t *__restrict__ k_cache, uint16_t *__restrict__ v_cache,
                   const int32_t *__restrict__ path, int max_path,
                   const int32_t *__restrict__ accept_len, int32_t *__restrict__ new_len) {
+    pdl_allow_dependents();
+    pdl_wait_predecessor();
     extern __shared__ uint4 stage[];      // [kCompactChunk][heads][D/8]
     __shared__ int s_src[kCompactChunk], s_dst[kCompactChunk];
     const int b = blockIdx.x;
@@ -91,10 +93,10 @@ cudaError_t launch_kv_compact(const BatchArgs &a, uint16_t *k_cache, uint16_t *v
                               int32_t *new_len, cudaStream_t st) {
     dim3 grid(a.B, 2, (a.Hkv + kHeadsPerCta - 1) / kHeadsPerCta);
     size_t smem = (size_t)kCompactChunk * kHeadsPerCta * (a.D / 8) * sizeof(uint4);
-    kv_compact_kernel<<<grid, kCompactThreads, smem, st>>>(a, k_cache, v_cache, path, max_path,
-                                                            accept_len, new_len);
+    cudaError_t e = launch_pdl(kv_compact_kernel, grid, dim3(kCompactThreads), smem, st, a, k_cache, v_cache, path,
+                               max_path, accept_len, new_len);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace jsv

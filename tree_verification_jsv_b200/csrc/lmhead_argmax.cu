@@ -100,6 +100,8 @@ template <int kSubTiles>
 __global__ void __launch_bounds__(LmShape<kSubTiles>::kThreads, 1)
 lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmW16,
                         const __grid_constant__ CUtensorMap tmH, const LmParams p) {
+    pdl_allow_dependents();
+    pdl_wait_predecessor();
     constexpr int kEpiWarps = LmShape<kSubTiles>::kEpiWarps;
     constexpr int kItemRows = LmShape<kSubTiles>::kItemRows;
     constexpr uint32_t kStageA = LmShape<kSubTiles>::kStageA;
@@ -397,11 +399,11 @@ cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int 
     if (grid <= 0) return cudaErrorInvalidDevice;
     if (grid > tiles) grid = tiles;
     if (sub == 1)
-        lmhead_argmax_tc_kernel<1><<<grid, LmShape<1>::kThreads, smem, st>>>(tmW, tmW16, tmH, p);
+        e = launch_pdl(lmhead_argmax_tc_kernel<1>, dim3(grid), dim3(LmShape<1>::kThreads), smem, st, tmW, tmW16, tmH, p);
     else
-        lmhead_argmax_tc_kernel<2><<<grid, LmShape<2>::kThreads, smem, st>>>(tmW, tmW16, tmH, p);
+        e = launch_pdl(lmhead_argmax_tc_kernel<2>, dim3(grid), dim3(LmShape<2>::kThreads), smem, st, tmW, tmW16, tmH, p);
     count_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace jsv

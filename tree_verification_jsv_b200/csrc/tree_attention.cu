@@ -91,6 +91,8 @@ template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const AttnParams prm) {
+    pdl_allow_dependents();
+    pdl_wait_predecessor();
     using L = AttnSmem<D>;
     constexpr int kHalves = D / 64;
     extern __shared__ uint8_t dsmem[];
@@ -575,6 +577,8 @@ template <int D>
 __global__ void __launch_bounds__(kCombineWarps * 32)
 tree_attention_combine_kernel(BatchArgs a, int S, const float *__restrict__ ws_o,
                               const float *__restrict__ ws_ml, uint16_t *__restrict__ out) {
+    pdl_allow_dependents();
+    pdl_wait_predecessor();
     constexpr int DPL = D / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
@@ -586,22 +590,39 @@ tree_attention_combine_kernel(BatchArgs a, int S, const float *__restrict__ ws_o
     const int i = rloc / G, h = g * G + rloc % G, t = r.base + i;
     const size_t row_id = (size_t)t * a.Hq + h;
     const size_t rows = (size_t)a.total_nodes * a.Hq;
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) {
-        const float l = ws_ml[((size_t)s * rows + row_id) * 2 + 1];
-        if (l > 0.f) M = fmaxf(M, ws_ml[((size_t)s * rows + row_id) * 2]);
+    // lane s holds split s's (max, sum); the merge weights come from warp
+    // reductions, so the partial loads below are independent of each other
+    float ms = -INFINITY, ls = 0.f;
+    if (lane < S) {
+        const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + ((size_t)lane * rows + row_id) * 2);
+        ms = ml.x;
+        ls = ml.y;
     }
-    float L = 0.f, o[DPL];
+    float M = ls > 0.f ? ms : -INFINITY;
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, sh));
+    const float cw = ls > 0.f ? exp2f(ms - M) : 0.f;
+    float L = ls * cw;
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) L += __shfl_xor_sync(0xffffffffu, L, sh);
+    float o[DPL];
 #pragma unroll
     for (int x = 0; x < DPL; ++x) o[x] = 0.f;
+#pragma unroll 4
     for (int s = 0; s < S; ++s) {
-        const float l = ws_ml[((size_t)s * rows + row_id) * 2 + 1];
-        if (!(l > 0.f)) continue;
-        const float c = exp2f(ws_ml[((size_t)s * rows + row_id) * 2] - M);
-        L = fmaf(l, c, L);
+        const float c = __shfl_sync(0xffffffffu, cw, s);
+        if (c == 0.f) continue;
         const float *po = ws_o + ((size_t)s * rows + row_id) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(po);
+            o[0] = fmaf(c, v.x, o[0]);
+            o[1] = fmaf(c, v.y, o[1]);
+            o[2] = fmaf(c, v.z, o[2]);
+            o[3] = fmaf(c, v.w, o[3]);
+        } else {
 #pragma unroll
-        for (int x = 0; x < DPL; ++x) o[x] = fmaf(c, po[x], o[x]);
+            for (int x = 0; x < DPL; ++x) o[x] = fmaf(c, po[x], o[x]);
+        }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     uint16_t *op = out + row_id * D + lane * DPL;
@@ -675,8 +696,7 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
         attr_set[dev] = true;
     }
     dim3 grid((a.max_nodes * G + kRowsPerCta - 1) / kRowsPerCta, S, a.B * a.Hkv);
-    tree_attention_tc_kernel<D><<<grid, kAttnThreads, smem, st>>>(tmK, tmV, prm);
-    cudaError_t le = cudaGetLastError();
+    cudaError_t le = launch_pdl(tree_attention_tc_kernel<D>, grid, dim3(kAttnThreads), smem, st, tmK, tmV, prm);
     if (le != cudaSuccess) {
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, tree_attention_tc_kernel<D>) == cudaSuccess)
@@ -685,9 +705,10 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
         return le;
     }
     dim3 cgrid((a.max_nodes * G + kCombineWarps - 1) / kCombineWarps, 1, a.B * a.Hkv);
-    tree_attention_combine_kernel<D><<<cgrid, kCombineWarps * 32, 0, st>>>(a, S, prm.ws_o, prm.ws_ml, out);
+    le = launch_pdl(tree_attention_combine_kernel<D>, cgrid, dim3(kCombineWarps * 32), 0, st, a, S,
+                    (const float *)prm.ws_o, (const float *)prm.ws_ml, out);
     count_launches(2);
-    return cudaGetLastError();
+    return le;
 }
 
 cudaError_t launch_tree_attention(const BatchArgs &a, const uint16_t *q, const uint16_t *k_cache,
