@@ -207,6 +207,18 @@ JSV_API jsv_status jsv_lmhead_argmax_noalloc(const uint16_t *hidden, const uint1
  * launches inside a timed region; not tied to any stream order. */
 JSV_API uint64_t jsv_kernel_launches(void);
 
+/*
+ * Failure-detection self-test of the bounded device waits.  Every wait of
+ * the library's tensor-core kernels on an mbarrier gives up after a time
+ * limit, writes JSV_ERR_TIMEOUT to the status word and unwinds (copies in
+ * flight drained, TMEM released), so a lost arrival ends in a readable status
+ * rather than a hung GPU.  This call launches one CTA that waits on a barrier
+ * nothing signals, with the limit shortened to `limit_us` microseconds
+ * (1 .. 2,000,000); it writes JSV_ERR_TIMEOUT to *dev_status (device int32,
+ * compare-and-swap from 0) and exits, leaving the context usable.
+ */
+JSV_API jsv_status jsv_selftest_wait_timeout(int32_t *dev_status, uint32_t limit_us, void *stream);
+
 /* Text of the last CUDA error behind a JSV_ERR_CUDA returned to the calling
  * host thread (a launch or runtime call that failed), or a fixed message if
  * none was recorded; for a failed kernel launch it also names the kernel's

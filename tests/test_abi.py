@@ -80,6 +80,10 @@ def test_host_validation_other_arguments(lib):
     assert lib.jsv_lmhead_argmax(16, 16, 4, 128, 50, 16, None, None, 0, None) == 1
     assert lib.jsv_lmhead_argmax(16, 16, 4, 128, 50, None, None, 16, 1 << 20, None) == 1
     assert lib.jsv_lmhead_argmax_workspace_size(4, 128, 50) >= 32
+    # bounded-wait self-test: NULL status word, limits out of range
+    assert lib.jsv_selftest_wait_timeout(None, 10, None) == 1
+    assert lib.jsv_selftest_wait_timeout(16, 0, None) == 1
+    assert lib.jsv_selftest_wait_timeout(16, 3_000_000, None) == 1
 
 
 def test_binding_raises_without_library(monkeypatch, tmp_path):

@@ -1,0 +1,37 @@
+"""The verify step captured in a CUDA graph gives the same bytes as the
+eager step (argmax, walk, compaction, attention output), on the tiny and
+the Qwen3-8B-shaped 64-node workloads."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import golden_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _bits(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["tiny", "8b_64"])
+def test_graph_replay_matches_eager_step(name):
+    from tree_verification_jsv_b200 import build
+    from tree_verification_jsv_b200.step import VerifyStep
+    build.build()
+    wl, tokens, _ = golden_workload(name)
+    eager = VerifyStep(wl, tokens)
+    eager.run()
+    torch.cuda.synchronize()
+
+    graphed = VerifyStep(wl, tokens)
+    k0, v0 = graphed.k_cache.clone(), graphed.v_cache.clone()
+    graphed.capture()                       # runs one eager step first
+    graphed.k_cache.copy_(k0)
+    graphed.v_cache.copy_(v0)
+    graphed.status.zero_()
+    graphed.replay()
+    torch.cuda.synchronize()
+    assert int(graphed.status.item()) == 0
+    for name_ in ("out", "argmax", "max_logit", "path", "accept_len", "bonus", "new_len", "k_cache", "v_cache"):
+        assert np.array_equal(_bits(getattr(eager, name_)), _bits(getattr(graphed, name_))), name_

@@ -23,7 +23,7 @@ JSV_ERR_DEVICE_INPUT = 5
 EXPORTS = ("jsv_tree_attention_workspace_size", "jsv_tree_attention",
            "jsv_lmhead_argmax_workspace_size", "jsv_lmhead_argmax", "jsv_accept_path",
            "jsv_kv_compact", "jsv_status_string", "jsv_version", "jsv_kernel_launches",
-           "jsv_lmhead_argmax_noalloc", "jsv_last_error_string")
+           "jsv_lmhead_argmax_noalloc", "jsv_last_error_string", "jsv_selftest_wait_timeout")
 
 # Largest node count jsv_lmhead_argmax_noalloc accepts (JSV_NOALLOC_MAX_NODES).
 NOALLOC_MAX_NODES = 8192
@@ -81,6 +81,8 @@ def load() -> ctypes.CDLL:
     lib.jsv_version.restype = i32
     lib.jsv_lmhead_argmax_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
     lib.jsv_lmhead_argmax_noalloc.restype = ctypes.c_int
+    lib.jsv_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
+    lib.jsv_selftest_wait_timeout.restype = ctypes.c_int
     lib.jsv_last_error_string.argtypes = []
     lib.jsv_last_error_string.restype = ctypes.c_char_p
     lib.jsv_kernel_launches.argtypes = []
@@ -166,6 +168,12 @@ def jsv_lmhead_argmax_noalloc(hidden, w, T, d, V, argmax, max_logit, stream=None
     st = load().jsv_lmhead_argmax_noalloc(_addr(hidden), _addr(w), int(T), int(d), int(V),
                                           _addr(argmax), _addr(max_logit), _stream(stream))
     _check("jsv_lmhead_argmax_noalloc", st)
+
+
+def jsv_selftest_wait_timeout(dev_status, limit_us, stream=None) -> None:
+    """Launch the bounded-wait self-test (see include/jsv.h)."""
+    st = load().jsv_selftest_wait_timeout(_addr(dev_status), int(limit_us), _stream(stream))
+    _check("jsv_selftest_wait_timeout", st)
 
 
 def jsv_accept_path(batch, tokens, argmax, max_path, path, accept_len, bonus, stream=None) -> None:

@@ -7,6 +7,11 @@ tree attention, LM head + argmax, accept walk, KV compaction.
 
 ``run_host`` is the end-to-end form: it copies the step's per-step inputs
 from pinned host memory, runs the step, and copies the accepted paths back.
+
+``capture`` records the four calls once into a CUDA graph (the engine the
+JetSpec README describes replays CUDA graphs for wall-clock latency); every
+kernel is launched with programmatic dependent launch, so the graph keeps
+those overlapping edges.  ``replay`` launches the whole step in one call.
 """
 from __future__ import annotations
 
@@ -64,6 +69,7 @@ class VerifyStep:
         self.attn_ws = torch.empty(max(aws, 256), dtype=torch.uint8, device=dev)
         self.lm_ws = torch.empty(max(lws, 8), dtype=torch.uint8, device=dev)
         self._pinned = None
+        self._graph = None
 
     # -- the four calls -----------------------------------------------------
     def attention(self, stream=None):
@@ -88,6 +94,27 @@ class VerifyStep:
         self.lmhead(stream)
         self.accept(stream)
         self.compact(stream)
+
+    # -- CUDA graph -----------------------------------------------------------
+    def capture(self):
+        """Record one verify step into a CUDA graph on a side stream.
+
+        One eager step runs first so that every one-time host set-up (kernel
+        attributes, tensor-map entry point) happens outside the capture; it
+        executes the step, so callers that need pristine caches restore them
+        before replaying."""
+        self.run()
+        torch.cuda.synchronize(self.device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.run()
+        torch.cuda.synchronize(self.device)
+        self._graph = graph
+        return graph
+
+    def replay(self):
+        """One verify step through the captured graph (same buffers)."""
+        self._graph.replay()
 
     # -- end-to-end form ----------------------------------------------------
     def host_inputs(self):
