@@ -248,3 +248,74 @@ def kv_compact(k_cache, v_cache, page_table, prefix_len, paths, page_size=16):
             v_cache[dp, do] = v_cache[sp, so]
         new_len.append(P + len(path))
     return np.asarray(new_len, dtype=np.int32)
+
+
+# ---------------------------------------------------------------------------
+# Budgeted tree construction by cumulative log-probability (accum_logp)
+# ---------------------------------------------------------------------------
+
+def accum_logp_tree(logp, topk_tokens, root_token, budget):
+    """The draft tree the pages' default ``accum_logp`` construction keeps
+    (JetSpec README, "Evaluation": a breadth-first tree kept by cumulative
+    log-probability under depth, width and budget).
+
+    Reading: the draft head gives, for each depth m = 1..D, its top-k
+    candidate tokens with log-probabilities sorted in descending order
+    (``logp[m-1][r]``, ``topk_tokens[m-1][r]``).  A node is a rank path
+    (r_1..r_m); its score is the fp32 running sum of its edge log-probs, added
+    root-to-leaf (the kernel's precision decides the comparison).  The tree
+    is the ``budget`` best nodes under the total order
+        score descending, then depth ascending, then the rank path read as a
+        base-k number ascending,
+    the root (empty path, score 0) included.  Children never outrank their
+    parent and a rank never outranks the previous rank, so that set is
+    ancestor- and sibling-closed.  It is returned in breadth-first order
+    (level by level, children by parent order then rank).
+
+    Best-first expansion visits nodes in exactly that order: a node enters
+    the candidate set when its parent (first child) or its previous sibling
+    is taken.  Returns dict(parent, tokens, depth, score, code) as numpy
+    arrays of length n <= budget."""
+    import heapq
+    logp = np.asarray(logp, dtype=np.float32)
+    topk_tokens = np.asarray(topk_tokens)
+    D, k = logp.shape
+    sel = [(-1, -1, 0, np.float32(0.0), 0)]        # (parent sel index, rank, depth, score, code)
+    heap = []
+
+    def push(parent_sel, rank, depth):
+        ps = sel[parent_sel][3]
+        s = np.float32(ps + logp[depth - 1][rank])
+        code = sel[parent_sel][4] * k + rank
+        heapq.heappush(heap, (-float(s), depth, code, parent_sel, rank, s))
+
+    if D >= 1 and k >= 1 and budget > 1:
+        push(0, 0, 1)
+    while heap and len(sel) < budget:
+        _, depth, code, parent_sel, rank, s = heapq.heappop(heap)
+        me = len(sel)
+        sel.append((parent_sel, rank, depth, s, code))
+        if rank + 1 < k:
+            push(parent_sel, rank + 1, depth)
+        if depth < D:
+            push(me, 0, depth + 1)
+    # breadth-first relabelling
+    n = len(sel)
+    kids = [[] for _ in range(n)]
+    for i in range(1, n):
+        kids[sel[i][0]].append(i)
+    for c in kids:
+        c.sort(key=lambda i: sel[i][1])
+    order = [0]
+    head = 0
+    while head < len(order):
+        order.extend(kids[order[head]])
+        head += 1
+    new = {old: new_i for new_i, old in enumerate(order)}
+    parent = np.array([-1] + [new[sel[o][0]] for o in order[1:]], dtype=np.int32)
+    depth = np.array([sel[o][2] for o in order], dtype=np.int32)
+    tokens = np.array([int(root_token)] + [int(topk_tokens[sel[o][2] - 1][sel[o][1]]) for o in order[1:]],
+                      dtype=np.int32)
+    score = np.array([sel[o][3] for o in order], dtype=np.float32)
+    code = np.array([sel[o][4] for o in order], dtype=np.uint64)
+    return dict(parent=parent, tokens=tokens, depth=depth, score=score, code=code)

@@ -352,3 +352,21 @@ def plant_tokens(wl: Workload, argmax: np.ndarray) -> np.ndarray:
             if wl.tok_flag[t]:
                 tok[t] = argmax[base + int(wl.parent[t])]
     return tok
+
+
+# --------------------------------------------------------------------------
+# Draft-head top-k per depth (input of the budgeted tree construction)
+# --------------------------------------------------------------------------
+
+def draft_topk(seed: int, B: int, D: int, k: int, V: int):
+    """Synthetic draft-head output for ``B`` requests: for each depth 1..D,
+    ``k`` candidate tokens with log-probabilities sorted in descending order
+    (logs of ``k`` normalised uniforms), plus a root token per request.
+    Returns (logp float32 [B][D][k], tokens int32 [B][D][k], root int32 [B])."""
+    g = _rng(seed, "tree", 10_000)
+    u = g.random((B, D, k)) + 1e-6
+    p = np.sort(u / u.sum(axis=2, keepdims=True), axis=2)[:, :, ::-1]
+    logp = np.log(p).astype(np.float32)
+    tok = g.integers(0, V, (B, D, k)).astype(np.int32)
+    root = g.integers(0, V, B).astype(np.int32)
+    return np.ascontiguousarray(logp), tok, root
