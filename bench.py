@@ -44,6 +44,12 @@ DESCRIPTION = {
     "30b_512x4": "Qwen3-30B-A3B-shaped: 32q/4kv, head_dim 128, hidden 2048, vocab 151936, batch 4, prefix 32768, 512-node trees (depth 16, top-8)",
 }
 
+# draft-tree shape of each workload for the tree-construction timing:
+# (depth, width, budget) -- the pages' tree_depth / tree_width / budget
+TREE_SHAPE = {"tiny": (5, 3, 16), "8b_64": (8, 4, 64), "8b_256": (16, 8, 256),
+              "ragged16": (12, 4, 128), "30b_512x4": (16, 8, 512)}
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -372,6 +378,33 @@ def run_gpu(args, rank, world, local_rank):
         assert int(st.status.item()) == 0
         graph = float(np.mean([a.elapsed_time(b) for a, b in evg]))
 
+    # tree construction (accum_logp) for this workload's tree shape, per request
+    tree_us = None
+    if not args.no_graph:
+        from tree_verification_jsv_b200 import synth as _synth
+        Dt, kt, bt = TREE_SHAPE[args.workload]
+        lp, tk, rt = _synth.draft_topk(wl.seed, wl.B, Dt, kt, wl.V)
+        dev = f"cuda:{local_rank}"
+        lp_d, tk_d, rt_d = (torch.as_tensor(x).to(dev) for x in (lp, tk, rt))
+        tp = torch.empty((wl.B, bt), dtype=torch.int32, device=dev)
+        ttok, tdep = torch.empty_like(tp), torch.empty_like(tp)
+        tsc = torch.empty((wl.B, bt), dtype=torch.float32, device=dev)
+        tnn = torch.empty(wl.B, dtype=torch.int32, device=dev)
+
+        def build_tree():
+            jsv.jsv_accum_logp_tree(lp_d, tk_d, rt_d, wl.B, Dt, kt, bt, tp, ttok, tdep, tsc, tnn, st.status)
+        for _ in range(3):
+            build_tree()
+        torch.cuda.synchronize()
+        et0, et1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        et0.record(stream)
+        for _ in range(K):
+            build_tree()
+        et1.record(stream)
+        torch.cuda.synchronize()
+        assert int(st.status.item()) == 0
+        tree_us = 1e3 * et0.elapsed_time(et1) / K
+
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -439,6 +472,10 @@ def run_gpu(args, rank, world, local_rank):
         "clocks": clocks.summary(),
         "accept_len": g["accept_len"][:16],
     }
+    if tree_us is not None:
+        Dt, kt, bt = TREE_SHAPE[args.workload]
+        line["tree_build"] = {"us_per_call": tree_us, "requests": wl.B, "depth": Dt, "width": kt, "budget": bt,
+                              "call": "jsv_accum_logp_tree (not part of the verify step)"}
     if graph:
         line["graph"] = {"value": whole_job_value(wl.T, world, graph_ms_max), "unit": "nodes/s",
                          "ms_per_step": graph_ms_max,

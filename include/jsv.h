@@ -120,6 +120,37 @@ JSV_API jsv_status jsv_tree_attention(const jsv_batch *batch, const uint16_t *q,
                               float scale, uint16_t *out,
                               void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Budgeted draft-tree construction by cumulative log-probability (the pages'
+ * default "accum_logp" tree: JetSpec README, "Evaluation", breadth-first and
+ * kept by cumulative log-probability under depth, width and budget).  Reading:
+ * for each request the draft head gives, per depth m = 1..depth, its top-width
+ * candidate tokens with log-probabilities sorted in descending order.  A node
+ * is a rank path; its score is the fp32 running sum of its edge log-probs
+ * (added root to leaf).  The tree is the `budget` best nodes under
+ *     score descending, depth ascending, rank path lexicographic ascending
+ * (root = empty path, score 0, always kept), in breadth-first order with
+ * children in rank order: parent[0] = -1 and parent[i] < i, ready for the
+ * other calls.
+ *   logp         device [B][depth][width] float, each row non-increasing, <= 0
+ *   topk_tokens  device [B][depth][width] int32
+ *   root_token   device [B] int32 (the last committed token)
+ *   parent, tokens, node_depth  device [B][budget] int32 outputs; slots past
+ *                num_nodes[b] get -1
+ *   score        device [B][budget] float or NULL (fp32 node scores)
+ *   num_nodes    device [B] int32: nodes emitted (budget, or fewer when the
+ *                whole candidate tree is smaller)
+ *   dev_status   device [1] int32 or NULL: a request whose log-probs are not
+ *                sorted, positive or NaN gets JSV_ERR_DEVICE_INPUT and a
+ *                root-only tree
+ * Supported: 1 <= B, 0 <= depth <= 32, 1 <= width <= 32, 1 <= budget <= 512.
+ */
+JSV_API jsv_status jsv_accum_logp_tree(const float *logp, const int32_t *topk_tokens,
+                                       const int32_t *root_token, int32_t B, int32_t depth,
+                                       int32_t width, int32_t budget, int32_t *parent,
+                                       int32_t *tokens, int32_t *node_depth, float *score,
+                                       int32_t *num_nodes, int32_t *dev_status, void *stream);
+
 /* Bytes of scratch jsv_lmhead_argmax needs (one 64-bit key per node and a
  * completion counter). */
 JSV_API size_t jsv_lmhead_argmax_workspace_size(int32_t T, int32_t d, int32_t V);

@@ -110,6 +110,19 @@ jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uint16_t *v
                                             accept_len, new_len, static_cast<cudaStream_t>(stream)));
 }
 
+jsv_status jsv_accum_logp_tree(const float *logp, const int32_t *topk_tokens, const int32_t *root_token,
+                               int32_t B, int32_t depth, int32_t width, int32_t budget, int32_t *parent,
+                               int32_t *tokens, int32_t *node_depth, float *score, int32_t *num_nodes,
+                               int32_t *dev_status, void *stream) {
+    if (B < 1 || depth < 0 || width < 1 || budget < 1) return JSV_ERR_INVALID_ARG;
+    if (depth > 32 || width > 32 || budget > 512) return JSV_ERR_UNSUPPORTED;
+    if ((depth > 0 && (!logp || !topk_tokens)) || !root_token || !parent || !tokens || !node_depth || !num_nodes)
+        return JSV_ERR_INVALID_ARG;
+    return from_cuda(jsv::launch_accum_logp_tree(logp, topk_tokens, root_token, B, depth, width, budget, parent,
+                                                 tokens, node_depth, score, num_nodes, dev_status,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
 const char *jsv_status_string(jsv_status status) {
     switch (status) {
         case JSV_OK: return "ok";

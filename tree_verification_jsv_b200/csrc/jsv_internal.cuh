@@ -119,6 +119,9 @@ size_t lmhead_workspace_bytes(int T, int d, int V);
 cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int T, int d, int V,
                                  int32_t *argmax, float *max_logit, void *ws, cudaStream_t st);
 size_t attention_workspace_bytes(const BatchArgs &a);
+cudaError_t launch_accum_logp_tree(const float *logp, const int32_t *topk_tokens, const int32_t *root_token, int B,
+                                   int D, int k, int budget, int32_t *parent, int32_t *tokens, int32_t *depth,
+                                   float *score, int32_t *num_nodes, int32_t *status, cudaStream_t st);
 cudaError_t launch_tree_attention(const BatchArgs &a, const uint16_t *q, const uint16_t *k_cache,
                                   const uint16_t *v_cache, float scale, uint16_t *out, void *ws,
                                   cudaStream_t st);

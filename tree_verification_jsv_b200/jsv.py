@@ -23,7 +23,8 @@ JSV_ERR_DEVICE_INPUT = 5
 EXPORTS = ("jsv_tree_attention_workspace_size", "jsv_tree_attention",
            "jsv_lmhead_argmax_workspace_size", "jsv_lmhead_argmax", "jsv_accept_path",
            "jsv_kv_compact", "jsv_status_string", "jsv_version", "jsv_kernel_launches",
-           "jsv_lmhead_argmax_noalloc", "jsv_last_error_string", "jsv_selftest_wait_timeout")
+           "jsv_lmhead_argmax_noalloc", "jsv_last_error_string", "jsv_selftest_wait_timeout",
+           "jsv_accum_logp_tree")
 
 # Largest node count jsv_lmhead_argmax_noalloc accepts (JSV_NOALLOC_MAX_NODES).
 NOALLOC_MAX_NODES = 8192
@@ -81,6 +82,8 @@ def load() -> ctypes.CDLL:
     lib.jsv_version.restype = i32
     lib.jsv_lmhead_argmax_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
     lib.jsv_lmhead_argmax_noalloc.restype = ctypes.c_int
+    lib.jsv_accum_logp_tree.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.jsv_accum_logp_tree.restype = ctypes.c_int
     lib.jsv_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
     lib.jsv_selftest_wait_timeout.restype = ctypes.c_int
     lib.jsv_last_error_string.argtypes = []
@@ -168,6 +171,14 @@ def jsv_lmhead_argmax_noalloc(hidden, w, T, d, V, argmax, max_logit, stream=None
     st = load().jsv_lmhead_argmax_noalloc(_addr(hidden), _addr(w), int(T), int(d), int(V),
                                           _addr(argmax), _addr(max_logit), _stream(stream))
     _check("jsv_lmhead_argmax_noalloc", st)
+
+
+def jsv_accum_logp_tree(logp, topk_tokens, root_token, B, depth, width, budget, parent, tokens,
+                        node_depth, score, num_nodes, dev_status=None, stream=None) -> None:
+    st = load().jsv_accum_logp_tree(_addr(logp), _addr(topk_tokens), _addr(root_token), int(B), int(depth),
+                                    int(width), int(budget), _addr(parent), _addr(tokens), _addr(node_depth),
+                                    _addr(score), _addr(num_nodes), _addr(dev_status), _stream(stream))
+    _check("jsv_accum_logp_tree", st)
 
 
 def jsv_selftest_wait_timeout(dev_status, limit_us, stream=None) -> None:
