@@ -319,3 +319,68 @@ def accum_logp_tree(logp, topk_tokens, root_token, budget):
     score = np.array([sel[o][3] for o in order], dtype=np.float32)
     code = np.array([sel[o][4] for o in order], dtype=np.uint64)
     return dict(parent=parent, tokens=tokens, depth=depth, score=score, code=code)
+
+
+# ---------------------------------------------------------------------------
+# Tree Q/K/V projection with rotary positions, K/V appended to the paged cache
+# ---------------------------------------------------------------------------
+
+def rope_rotate(x, cos, sin):
+    """Rotate-half rotary embedding of one head vector x (length D) with the
+    pair tables cos/sin (length D/2): out_i = x_i c_i - x_{i+D/2} s_i and
+    out_{i+D/2} = x_{i+D/2} c_i + x_i s_i."""
+    h = len(x) // 2
+    a, b = x[:h], x[h:]
+    return np.concatenate([a * cos - b * sin, b * cos + a * sin])
+
+
+def tree_qkv_rope(*, x, w_qkv, Hq, Hkv, D, page_table, prefix_len, node_offsets, parent,
+                  rope_cos, rope_sin, k_cache, v_cache, page_size=16):
+    """The step on the other side of the tree attention (reading of the JetSpec
+    README, "JetSpec / Overview" and "Quick Start": one forward over the tree
+    with a paged KV cache).  For node j of request b: qkv = W_qkv x_j (fp64;
+    rows Q heads, then K heads, then V heads); Q and K heads are rotated at
+    position P_b + depth(j) (a node sits one position after its parent); K and
+    V heads are written to logical slot P_b + j of the request's pages.
+    Returns q as float64 [T][Hq][D]; k_cache/v_cache (uint16 bf16 bits) are
+    updated in place with the fp64 K/V rounded to bf16 (nearest-even)."""
+    X = bf16_to_f64(x)
+    W = bf16_to_f64(w_qkv)
+    T = X.shape[0]
+    Y = X @ W.T                                   # [T][(Hq + 2 Hkv) D]
+    q = np.zeros((T, Hq, D))
+    cos = np.asarray(rope_cos, dtype=np.float64)
+    sin = np.asarray(rope_sin, dtype=np.float64)
+    kc = np.zeros((T, Hkv, D))
+    vc = np.zeros((T, Hkv, D))
+    for b in range(len(node_offsets) - 1):
+        s0, s1 = int(node_offsets[b]), int(node_offsets[b + 1])
+        P = int(prefix_len[b])
+        par = np.asarray(parent[s0:s1])
+        depth = np.zeros(s1 - s0, dtype=np.int64)
+        for i in range(1, s1 - s0):
+            depth[i] = depth[par[i]] + 1
+        for i in range(s1 - s0):
+            t = s0 + i
+            pos = P + int(depth[i])
+            for h in range(Hq):
+                q[t, h] = rope_rotate(Y[t, h * D:(h + 1) * D], cos[pos], sin[pos])
+            for g in range(Hkv):
+                off = (Hq + g) * D
+                kc[t, g] = rope_rotate(Y[t, off:off + D], cos[pos], sin[pos])
+                off = (Hq + Hkv + g) * D
+                vc[t, g] = Y[t, off:off + D]
+            slot = P + i
+            pg, ro = int(page_table[b, slot // page_size]), slot % page_size
+            k_cache[pg, ro] = _f64_to_bf16_bits(kc[t])
+            v_cache[pg, ro] = _f64_to_bf16_bits(vc[t])
+    return q, kc, vc
+
+
+def _f64_to_bf16_bits(a):
+    """Round float64 values to nearest-even bf16 through fp32 (round to fp32
+    first, then to bf16) -- only used to place oracle values in a bf16 cache."""
+    f = np.asarray(a, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u >> 16) & 1) + 0x7FFF
+    return ((u + r) >> 16).astype(np.uint16)
