@@ -21,6 +21,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -405,6 +406,37 @@ def run_gpu(args, rank, world, local_rank):
         assert int(st.status.item()) == 0
         tree_us = 1e3 * et0.elapsed_time(et1) / K
 
+    # tree Q/K/V projection + rotary + paged K/V append (the step before the attention)
+    qkv = None
+    if not args.no_graph:
+        from tree_verification_jsv_b200 import rope as _rope
+        dev = f"cuda:{local_rank}"
+        rows = (wl.Hq + 2 * wl.Hkv) * wl.D
+        gq = torch.Generator(device=dev).manual_seed(wl.seed)
+        w_qkv = (torch.randn(rows, wl.d, device=dev, generator=gq) / math.sqrt(wl.d)).to(torch.bfloat16)
+        max_pos = wl.max_prefix + wl.max_nodes + 1
+        cos_t, sin_t = (torch.as_tensor(t).to(dev) for t in _rope.rope_tables(1e6, wl.D, max_pos))
+
+        def qkv_call():
+            jsv.jsv_tree_qkv_rope(st.batch, st.hidden, w_qkv, wl.d, cos_t, sin_t, max_pos, st.q,
+                                  st.k_cache, st.v_cache)
+        for _ in range(3):
+            qkv_call()
+        torch.cuda.synchronize()
+        evq = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            evq[i][0].record(stream)
+            qkv_call()
+            evq[i][1].record(stream)
+        torch.cuda.synchronize()
+        assert int(st.status.item()) == 0
+        q_us = 1e3 * float(np.mean([a_.elapsed_time(b_) for a_, b_ in evq]))
+        q_bytes = rows * wl.d * 2 + wl.T * wl.d * 2 + wl.T * rows * 2
+        qkv = {"us_per_call": q_us, "algorithmic_bytes": q_bytes,
+               "achieved_gbs": q_bytes / (q_us * 1e-6) / 1e9,
+               "call": "jsv_tree_qkv_rope (the projection feeding the verify step; not timed in it)"}
+
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -472,6 +504,9 @@ def run_gpu(args, rank, world, local_rank):
         "clocks": clocks.summary(),
         "accept_len": g["accept_len"][:16],
     }
+    if qkv is not None:
+        qkv["frac_of_hbm_peak"] = qkv["achieved_gbs"] / hbm
+        line["qkv_rope"] = qkv
     if tree_us is not None:
         Dt, kt, bt = TREE_SHAPE[args.workload]
         line["tree_build"] = {"us_per_call": tree_us, "requests": wl.B, "depth": Dt, "width": kt, "budget": bt,

@@ -151,6 +151,30 @@ JSV_API jsv_status jsv_accum_logp_tree(const float *logp, const int32_t *topk_to
                                        int32_t *tokens, int32_t *node_depth, float *score,
                                        int32_t *num_nodes, int32_t *dev_status, void *stream);
 
+/*
+ * Tree Q/K/V projection with rotary positions, K/V appended to the paged cache
+ * (the step before jsv_tree_attention; reading of the JetSpec README,
+ * "JetSpec / Overview" and "Quick Start": one forward pass over the tree,
+ * paged KV).  For node j of request b, qkv = w_qkv x_j with rows Q heads
+ * (Hq*D), then K heads (Hkv*D), then V heads (Hkv*D); Q and K heads are
+ * rotated at position P_b + depth(j) with the rotate-half pairs (i, i + D/2):
+ *     out_i = x_i c_i - x_{i+D/2} s_i,  out_{i+D/2} = x_{i+D/2} c_i + x_i s_i
+ * Q is written to q[j], K and V to logical slot P_b + j of the request's
+ * pages.  fp32 accumulation, bf16 outputs.
+ *   x          device [T][d] bf16 (the tree's hidden states entering the layer)
+ *   w_qkv      device [(Hq + 2 Hkv) D][d] bf16
+ *   rope_cos, rope_sin  device [max_pos][D/2] float tables
+ *   q          device [T][Hq][D] bf16 output
+ *   k_cache, v_cache  the paged caches; only tree slots P_b .. P_b+N_b-1 change
+ * A node whose position reaches max_pos, or whose parent chain or page is
+ * malformed, is skipped and JSV_ERR_DEVICE_INPUT is written to dev_status.
+ * Supported: d % 64 == 0, 64 <= d <= 16384.
+ */
+JSV_API jsv_status jsv_tree_qkv_rope(const jsv_batch *batch, const uint16_t *x, const uint16_t *w_qkv,
+                                     int32_t d, const float *rope_cos, const float *rope_sin,
+                                     int32_t max_pos, uint16_t *q, uint16_t *k_cache,
+                                     uint16_t *v_cache, void *stream);
+
 /* Bytes of scratch jsv_lmhead_argmax needs (one 64-bit key per node and a
  * completion counter). */
 JSV_API size_t jsv_lmhead_argmax_workspace_size(int32_t T, int32_t d, int32_t V);

@@ -11,7 +11,7 @@ CSRC = PKG / "csrc"
 SO = PKG / "libjsv.so"
 SOURCES = ["jsv_api.cu", "tree_attention.cu", "lmhead_argmax.cu", "accept_path.cu", "kv_compact.cu",
            "lmhead_noalloc.cu", "tma_host.cu", "selftest.cu",
-           "tree_build.cu"]
+           "tree_build.cu", "qkv_rope.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

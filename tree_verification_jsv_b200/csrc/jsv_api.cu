@@ -110,6 +110,20 @@ jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uint16_t *v
                                             accept_len, new_len, static_cast<cudaStream_t>(stream)));
 }
 
+jsv_status jsv_tree_qkv_rope(const jsv_batch *batch, const uint16_t *x, const uint16_t *w_qkv, int32_t d,
+                             const float *rope_cos, const float *rope_sin, int32_t max_pos, uint16_t *q,
+                             uint16_t *k_cache, uint16_t *v_cache, void *stream) {
+    jsv_status s = check_batch(batch);
+    if (s != JSV_OK) return s;
+    if (!x || !w_qkv || !rope_cos || !rope_sin || !q || !k_cache || !v_cache || max_pos < 1 || d < 1)
+        return JSV_ERR_INVALID_ARG;
+    if (d % 64 != 0 || d > 16384) return JSV_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+        return JSV_ERR_INVALID_ARG;
+    return from_cuda(jsv::launch_tree_qkv_rope(jsv::to_args(batch), x, w_qkv, d, rope_cos, rope_sin, max_pos, q,
+                                               k_cache, v_cache, static_cast<cudaStream_t>(stream)));
+}
+
 jsv_status jsv_accum_logp_tree(const float *logp, const int32_t *topk_tokens, const int32_t *root_token,
                                int32_t B, int32_t depth, int32_t width, int32_t budget, int32_t *parent,
                                int32_t *tokens, int32_t *node_depth, float *score, int32_t *num_nodes,

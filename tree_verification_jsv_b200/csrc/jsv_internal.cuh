@@ -119,6 +119,9 @@ size_t lmhead_workspace_bytes(int T, int d, int V);
 cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int T, int d, int V,
                                  int32_t *argmax, float *max_logit, void *ws, cudaStream_t st);
 size_t attention_workspace_bytes(const BatchArgs &a);
+cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const uint16_t *w_qkv, int d,
+                                 const float *rope_cos, const float *rope_sin, int max_pos, uint16_t *q,
+                                 uint16_t *k_cache, uint16_t *v_cache, cudaStream_t st);
 cudaError_t launch_accum_logp_tree(const float *logp, const int32_t *topk_tokens, const int32_t *root_token, int B,
                                    int D, int k, int budget, int32_t *parent, int32_t *tokens, int32_t *depth,
                                    float *score, int32_t *num_nodes, int32_t *status, cudaStream_t st);

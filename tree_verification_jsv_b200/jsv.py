@@ -24,7 +24,7 @@ EXPORTS = ("jsv_tree_attention_workspace_size", "jsv_tree_attention",
            "jsv_lmhead_argmax_workspace_size", "jsv_lmhead_argmax", "jsv_accept_path",
            "jsv_kv_compact", "jsv_status_string", "jsv_version", "jsv_kernel_launches",
            "jsv_lmhead_argmax_noalloc", "jsv_last_error_string", "jsv_selftest_wait_timeout",
-           "jsv_accum_logp_tree")
+           "jsv_accum_logp_tree", "jsv_tree_qkv_rope")
 
 # Largest node count jsv_lmhead_argmax_noalloc accepts (JSV_NOALLOC_MAX_NODES).
 NOALLOC_MAX_NODES = 8192
@@ -82,6 +82,8 @@ def load() -> ctypes.CDLL:
     lib.jsv_version.restype = i32
     lib.jsv_lmhead_argmax_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
     lib.jsv_lmhead_argmax_noalloc.restype = ctypes.c_int
+    lib.jsv_tree_qkv_rope.argtypes = [bp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp]
+    lib.jsv_tree_qkv_rope.restype = ctypes.c_int
     lib.jsv_accum_logp_tree.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp]
     lib.jsv_accum_logp_tree.restype = ctypes.c_int
     lib.jsv_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
@@ -171,6 +173,14 @@ def jsv_lmhead_argmax_noalloc(hidden, w, T, d, V, argmax, max_logit, stream=None
     st = load().jsv_lmhead_argmax_noalloc(_addr(hidden), _addr(w), int(T), int(d), int(V),
                                           _addr(argmax), _addr(max_logit), _stream(stream))
     _check("jsv_lmhead_argmax_noalloc", st)
+
+
+def jsv_tree_qkv_rope(batch, x, w_qkv, d, rope_cos, rope_sin, max_pos, q, k_cache, v_cache,
+                      stream=None) -> None:
+    st = load().jsv_tree_qkv_rope(ctypes.byref(batch), _addr(x), _addr(w_qkv), int(d), _addr(rope_cos),
+                                  _addr(rope_sin), int(max_pos), _addr(q), _addr(k_cache), _addr(v_cache),
+                                  _stream(stream))
+    _check("jsv_tree_qkv_rope", st)
 
 
 def jsv_accum_logp_tree(logp, topk_tokens, root_token, B, depth, width, budget, parent, tokens,
