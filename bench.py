@@ -61,9 +61,44 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
-    ap.add_argument("--profile", choices=["attention", "lmhead", "accept", "compact"],
+    ap.add_argument("--profile", choices=["attention", "lmhead", "accept", "compact", "tree", "qkv"],
                     help="run only this call K times after W warm-up (for ncu); prints its mean time")
     return ap.parse_args()
+
+
+def tree_call(wl, st, dev):
+    """A jsv_accum_logp_tree call on this workload's draft-tree shape (seeded top-k)."""
+    import torch
+    from tree_verification_jsv_b200 import jsv
+    from tree_verification_jsv_b200 import synth as _synth
+    Dt, kt, bt = TREE_SHAPE[wl.name]
+    lp, tk, rt = _synth.draft_topk(wl.seed, wl.B, Dt, kt, wl.V)
+    lp_d, tk_d, rt_d = (torch.as_tensor(x).to(dev) for x in (lp, tk, rt))
+    tp = torch.empty((wl.B, bt), dtype=torch.int32, device=dev)
+    ttok, tdep = torch.empty_like(tp), torch.empty_like(tp)
+    tsc = torch.empty((wl.B, bt), dtype=torch.float32, device=dev)
+    tnn = torch.empty(wl.B, dtype=torch.int32, device=dev)
+
+    def call():
+        jsv.jsv_accum_logp_tree(lp_d, tk_d, rt_d, wl.B, Dt, kt, bt, tp, ttok, tdep, tsc, tnn, st.status)
+    return call
+
+
+def qkv_rope_call(wl, st, dev):
+    """A jsv_tree_qkv_rope call: seeded random-init fused Q/K/V weights, rotary base 1e6."""
+    import torch
+    from tree_verification_jsv_b200 import jsv
+    from tree_verification_jsv_b200 import rope as _rope
+    rows = (wl.Hq + 2 * wl.Hkv) * wl.D
+    gq = torch.Generator(device=dev).manual_seed(wl.seed)
+    w_qkv = (torch.randn(rows, wl.d, device=dev, generator=gq) / math.sqrt(wl.d)).to(torch.bfloat16)
+    max_pos = wl.max_prefix + wl.max_nodes + 1
+    cos_t, sin_t = (torch.as_tensor(t).to(dev) for t in _rope.rope_tables(1e6, wl.D, max_pos))
+
+    def call():
+        jsv.jsv_tree_qkv_rope(st.batch, st.hidden, w_qkv, wl.d, cos_t, sin_t, max_pos, st.q,
+                              st.k_cache, st.v_cache)
+    return call
 
 
 def golden(name):
@@ -293,7 +328,12 @@ def run_gpu(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
 
     if args.profile:
-        call = getattr(st, args.profile)
+        if args.profile == "tree":
+            call = tree_call(wl, st, f"cuda:{local_rank}")
+        elif args.profile == "qkv":
+            call = qkv_rope_call(wl, st, f"cuda:{local_rank}")
+        else:
+            call = getattr(st, args.profile)
         for _ in range(args.warmup):
             call()
         torch.cuda.synchronize()
@@ -382,18 +422,8 @@ def run_gpu(args, rank, world, local_rank):
     # tree construction (accum_logp) for this workload's tree shape, per request
     tree_us = None
     if not args.no_graph:
-        from tree_verification_jsv_b200 import synth as _synth
         Dt, kt, bt = TREE_SHAPE[args.workload]
-        lp, tk, rt = _synth.draft_topk(wl.seed, wl.B, Dt, kt, wl.V)
-        dev = f"cuda:{local_rank}"
-        lp_d, tk_d, rt_d = (torch.as_tensor(x).to(dev) for x in (lp, tk, rt))
-        tp = torch.empty((wl.B, bt), dtype=torch.int32, device=dev)
-        ttok, tdep = torch.empty_like(tp), torch.empty_like(tp)
-        tsc = torch.empty((wl.B, bt), dtype=torch.float32, device=dev)
-        tnn = torch.empty(wl.B, dtype=torch.int32, device=dev)
-
-        def build_tree():
-            jsv.jsv_accum_logp_tree(lp_d, tk_d, rt_d, wl.B, Dt, kt, bt, tp, ttok, tdep, tsc, tnn, st.status)
+        build_tree = tree_call(wl, st, f"cuda:{local_rank}")
         for _ in range(3):
             build_tree()
         torch.cuda.synchronize()
@@ -409,17 +439,8 @@ def run_gpu(args, rank, world, local_rank):
     # tree Q/K/V projection + rotary + paged K/V append (the step before the attention)
     qkv = None
     if not args.no_graph:
-        from tree_verification_jsv_b200 import rope as _rope
-        dev = f"cuda:{local_rank}"
         rows = (wl.Hq + 2 * wl.Hkv) * wl.D
-        gq = torch.Generator(device=dev).manual_seed(wl.seed)
-        w_qkv = (torch.randn(rows, wl.d, device=dev, generator=gq) / math.sqrt(wl.d)).to(torch.bfloat16)
-        max_pos = wl.max_prefix + wl.max_nodes + 1
-        cos_t, sin_t = (torch.as_tensor(t).to(dev) for t in _rope.rope_tables(1e6, wl.D, max_pos))
-
-        def qkv_call():
-            jsv.jsv_tree_qkv_rope(st.batch, st.hidden, w_qkv, wl.d, cos_t, sin_t, max_pos, st.q,
-                                  st.k_cache, st.v_cache)
+        qkv_call = qkv_rope_call(wl, st, f"cuda:{local_rank}")
         for _ in range(3):
             qkv_call()
         torch.cuda.synchronize()

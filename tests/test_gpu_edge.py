@@ -1,6 +1,7 @@
 """GPU edge cases through the C ABI: tiny and degenerate trees, ragged
 prefixes that are not multiples of the page size, trees crossing page
-boundaries, sharp attention, head-dim 64, G = 1, vocabulary and node counts
+boundaries, sharp attention, head-dim 64, G = 1 and G that does not divide a
+row group, vocabulary and node counts
 that are not tile multiples, and device-side error reporting."""
 import math
 
@@ -71,6 +72,11 @@ ATTN_CASES = {
     "head_dim_64_g1": ([synth.tiny_tree(np.random.default_rng(3), 31, 5, 3)], [45], 4, 4, 64),
     "g8_long": ([synth.budget_tree(np.random.default_rng(4), 100, 10, 4)], [1500], 16, 2, 128),
     "max_nodes_512": ([synth.budget_tree(np.random.default_rng(5), 512, 16, 8)], [64], 2, 1, 64),
+    # G that does not divide a 128-row group (Q staged by plain loads, rows
+    # of one node split across CTA tiles)
+    "g5_two_row_tiles": ([synth.budget_tree(np.random.default_rng(6), 60, 8, 4)], [700], 10, 2, 128),
+    "g3_head_dim_64": ([synth.tiny_tree(np.random.default_rng(7), 50, 6, 3),
+                        synth.tiny_tree(np.random.default_rng(8), 9, 3, 2)], [130, 33], 6, 2, 64),
 }
 
 

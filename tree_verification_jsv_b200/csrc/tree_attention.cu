@@ -38,6 +38,7 @@
 #include "sm100.cuh"
 
 #include <math.h>
+#include <string.h>
 
 namespace jsv {
 
@@ -68,6 +69,7 @@ struct AttnParams {
     const uint16_t *q;
     float scale_log2;
     int S;                 // splits
+    int q_tma;             // 1: Q is copied by TMA (G divides 128), 0: by the softmax warps
     float *ws_o;           // [S][T*Hq][D]
     float *ws_ml;          // [S][T*Hq][2]
 };
@@ -90,7 +92,7 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                         const AttnParams prm) {
+                         const __grid_constant__ CUtensorMap tmQ, const AttnParams prm) {
     pdl_allow_dependents();
     pdl_wait_predecessor();
     using L = AttnSmem<D>;
@@ -100,8 +102,8 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     __shared__ __align__(8) uint64_t s_full[kGroups], p_full[kGroups], o_done[kGroups], q_ready, drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
-    __shared__ volatile int sm_fail;
     __shared__ uint32_t anc[kRowsPerCta][kMaxTreeWords];
+    __shared__ int par_sh[32 * kMaxTreeWords];
 
     const BatchArgs &a = prm.a;
     const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
@@ -143,10 +145,9 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             mbar_init(&p_full[s], 4);
             mbar_init(&o_done[s], 1);
         }
-        mbar_init(&q_ready, 4 * kGroups);
+        mbar_init(&q_ready, 4 * kGroups + 1);     // softmax warps + the producer
         mbar_init(&drain_bar, 1);
         abort_sh = 0;
-        sm_fail = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -167,34 +168,55 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         // ----------------------------------------------------------- producer
         // The whole warp runs the loop: lanes 0..7 look up the 8 physical pages
         // of the NEXT tile (independent loads, issued before waiting for a free
-        // stage); lane 0 issues the copies, receiving page numbers by shuffle.
+        // stage) and each issues the copies of its own page.
         if (ntiles > 0) {
             if (lane == 0) {
+                // Q first: one box of 128 rows (128/G nodes x G heads) x 64 dims
+                // per row group and 64-dim block; rows past the request hold
+                // other nodes' (or zero-filled) queries and are never written out
+                if (prm.q_tma) {
+                    prefetch_tensormap(&tmQ);
+                    mbar_arrive_expect_tx(&q_ready, ngroups * L::kQGroupBytes);
+                    for (int grp = 0; grp < ngroups; ++grp) {
+                        const int node0 = r.base + (m0 + grp * kGroupRows) / G;
+#pragma unroll
+                        for (int h = 0; h < kHalves; ++h)
+                            tma_load_3d(sQ + grp * L::kQGroupBytes + h * (kGroupRows * 128), &tmQ, &q_ready, h * 64,
+                                        g * G, node0);
+                    }
+                } else {
+                    mbar_arrive(&q_ready);
+                }
                 prefetch_tensormap(&tmK);
                 prefetch_tensormap(&tmV);
             }
             const int oob = a.num_pages * a.page_size;   // fully out-of-bounds slot coordinate
             const int mapped_pages = (r.P + r.n + a.page_size - 1) / a.page_size;
-            auto lookup = [&](int j) -> int {            // slot coordinate of page `lane` of tile j
-                int z = oob;
+            // The page-table entry of page `lane` of tile j is loaded one tile
+            // ahead and checked only when that tile is issued, so the load does
+            // not hold up the copies of the current tile.
+            auto load_page = [&](int j) -> int {         // raw entry; -2: past the mapped pages
+                int page = -2;
                 if (lane < kKeyTile / 16) {
                     const int lp = tile_slot0(j) / 16 + lane;
-                    if (lp < mapped_pages) {
-                        const int page = a.page_table[(size_t)b * a.max_pages_per_req + lp];
-                        if (page >= 0 && page < a.num_pages) z = page * a.page_size;
-                        else flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
-                    }
+                    if (lp < mapped_pages) page = __ldg(a.page_table + (size_t)b * a.max_pages_per_req + lp);
                 }
-                return z;
+                return page;
+            };
+            auto to_slot = [&](int page) -> int {        // slot coordinate of a raw entry
+                if (page == -2) return oob;
+                if (page >= 0 && page < a.num_pages) return page * a.page_size;
+                flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+                return oob;
             };
             long long issued = 0;
             int stage = 0;
             uint32_t phase = 0;
-            int z_next = lookup(0);
+            int page_next = load_page(0);
             bool last_v_issued = true;
             for (int j = 0; j < ntiles; ++j) {
-                const int z_cur = z_next;
-                if (j + 1 < ntiles) z_next = lookup(j + 1);
+                const int z_cur = to_slot(page_next);
+                if (j + 1 < ntiles) page_next = load_page(j + 1);
                 // K of a stage frees once both groups' S of its previous tile are
                 // done, V once both groups' PV are
                 int ok = 1;
@@ -210,14 +232,11 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 uint8_t *sK = sKV + stage * L::kStageBytes;
                 uint8_t *sV = sK + L::kKVBytes;
                 if (lane == 0) mbar_arrive_expect_tx(&k_full[stage], L::kKVBytes);
+                __syncwarp();
+                if (lane < kKeyTile / 16) {
 #pragma unroll
-                for (int pg = 0; pg < kKeyTile / 16; ++pg) {
-                    const int z = __shfl_sync(0xffffffffu, z_cur, pg);
-                    if (lane == 0) {
-#pragma unroll
-                        for (int h = 0; h < kHalves; ++h)
-                            tma_load_3d(sK + h * (kKeyTile * 128) + pg * 2048, &tmK, &k_full[stage], h * 64, g, z);
-                    }
+                    for (int h = 0; h < kHalves; ++h)
+                        tma_load_3d(sK + h * (kKeyTile * 128) + lane * 2048, &tmK, &k_full[stage], h * 64, g, z_cur);
                 }
                 if (lane == 0) ok = mbar_wait(&v_empty[stage], phase ^ 1, &abort_sh) ? 1 : 0;
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -232,18 +251,19 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     break;
                 }
                 if (lane == 0) mbar_arrive_expect_tx(&v_full[stage], L::kKVBytes);
+                __syncwarp();
+                if (lane < kKeyTile / 16) {
 #pragma unroll
-                for (int pg = 0; pg < kKeyTile / 16; ++pg) {
-                    const int z = __shfl_sync(0xffffffffu, z_cur, pg);
-                    if (lane == 0) {
-#pragma unroll
-                        for (int h = 0; h < kHalves; ++h)
-                            tma_load_3d(sV + h * (kKeyTile * 128) + pg * 2048, &tmV, &v_full[stage], h * 64, g, z);
-                    }
+                    for (int h = 0; h < kHalves; ++h)
+                        tma_load_3d(sV + h * (kKeyTile * 128) + lane * 2048, &tmV, &v_full[stage], h * 64, g, z_cur);
                 }
                 ++issued;
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
                 if (abort_sh) break;
+            }
+            if (lane == 0 && prm.q_tma) {
+                int zero = 0;              // the Q copy has landed (long since, unless aborting)
+                mbar_wait(&q_ready, 0, (volatile int *)&zero);
             }
             if (lane == 0 && abort_sh) {
                 int zero = 0;
@@ -344,37 +364,82 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         const int node = rg / G;                     // request-local node
         const int head = g * G + rg % G;
 
-        // Q of both groups: rows x D bf16 in the K-major SW128 layout (zero rows past the end)
-        for (int e = et; e < kRowsPerCta * (D / 8); e += kGroups * 128) {
-            const int rr = e / (D / 8), c = e % (D / 8);
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (rr < rows_here) {
-                const int rgg = m0 + rr;
-                const uint16_t *src = prm.q + ((size_t)(r.base + rgg / G) * a.Hq + g * G + rgg % G) * D + c * 8;
-                v = *reinterpret_cast<const uint4 *>(src);
-            }
-            *reinterpret_cast<uint4 *>(sQ + (rr / kGroupRows) * L::kQGroupBytes + (c >> 3) * (kGroupRows * 128) +
-                                       sw128_offset(rr % kGroupRows, c & 7)) = v;
+        // With Q copied by TMA these warps take no part in it: they arrive at
+        // once.  Otherwise they load Q here: rows x D bf16 in the K-major SW128
+        // layout (zero rows past the end).  A thread issues a batch of loads
+        // before storing any of them, so that they overlap (one memory round
+        // trip per batch, not one per 16 bytes).
+        if (prm.q_tma) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_ready);
         }
-        // ancestor-or-self bitsets of this tile's rows (only the last split uses them)
+        constexpr int kParIters = 32 * kMaxTreeWords / (kGroups * 128);
+        int pv[kParIters];
+        if (tree_tiles > 0) {           // the request's parent array, for the tree mask
+#pragma unroll
+            for (int it = 0; it < kParIters; ++it) {
+                const int i = et + it * (kGroups * 128);
+                pv[it] = i < r.n ? __ldg(a.parent + r.base + i) : -1;
+            }
+        }
+        if (!prm.q_tma) {
+            constexpr int kQIters = kRowsPerCta * (D / 8) / (kGroups * 128);
+            constexpr int kQBatch = kQIters < 8 ? kQIters : 8;  // loads in flight per thread
+#pragma unroll
+            for (int i0 = 0; i0 < kQIters; i0 += kQBatch) {
+                uint4 qv[kQBatch];
+#pragma unroll
+                for (int it = 0; it < kQBatch; ++it) {
+                    const int e = et + (i0 + it) * (kGroups * 128);
+                    const int rr = e / (D / 8), c = e % (D / 8);
+                    qv[it] = make_uint4(0, 0, 0, 0);
+                    if (rr < rows_here) {
+                        const int rgg = m0 + rr;
+                        const uint16_t *src =
+                            prm.q + ((size_t)(r.base + rgg / G) * a.Hq + g * G + rgg % G) * D + c * 8;
+                        qv[it] = __ldg(reinterpret_cast<const uint4 *>(src));
+                    }
+                }
+#pragma unroll
+                for (int it = 0; it < kQBatch; ++it) {
+                    const int e = et + (i0 + it) * (kGroups * 128);
+                    const int rr = e / (D / 8), c = e % (D / 8);
+                    *reinterpret_cast<uint4 *>(sQ + (rr / kGroupRows) * L::kQGroupBytes +
+                                               (c >> 3) * (kGroupRows * 128) + sw128_offset(rr % kGroupRows, c & 7)) =
+                        qv[it];
+                }
+            }
+            fence_async_smem();
+        }
+        if (tree_tiles > 0) {
+#pragma unroll
+            for (int it = 0; it < kParIters; ++it) par_sh[et + it * (kGroups * 128)] = pv[it];
+        }
+        if (tree_tiles > 0 || !prm.q_tma) named_barrier(1, kGroups * 128);
+        if (!prm.q_tma) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_ready);
+        }
+        // ancestor-or-self bitsets of this tile's rows (only the CTA that covers
+        // the tree slots uses them), walked over the parent array in shared
+        // memory; each thread reads and writes only its own row's bitset
         if (tree_tiles > 0 && row_valid) {
             for (int w = 0; w < kMaxTreeWords; ++w) anc[row][w] = 0;
             int j = node, steps = 0;
             while (j != -1) {
-                if (steps++ > r.n || j >= 32 * kMaxTreeWords) { sm_fail = 1; break; }
+                if (steps++ > r.n || j >= 32 * kMaxTreeWords) {
+                    flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+                    break;
+                }
                 anc[row][j >> 5] |= 1u << (j & 31);
-                const int p = a.parent[r.base + j];
-                if (j == 0 ? p != -1 : (p < 0 || p >= j)) { sm_fail = 1; break; }
+                const int p = par_sh[j];
+                if (j == 0 ? p != -1 : (p < 0 || p >= j)) {
+                    flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
+                    break;
+                }
                 j = p;
             }
         }
-        fence_async_smem();
-        named_barrier(1, kGroups * 128);
-        if (sm_fail) {
-            if (et == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&q_ready);
 
         float m_used = -INFINITY, l = 0.f;
         const float sl2 = prm.scale_log2;
@@ -535,24 +600,44 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         }
         const size_t rows = (size_t)a.total_nodes * a.Hq;
         const size_t row_id = (size_t)(r.base + min(node, r.n - 1)) * a.Hq + head;
-        float4 *po = reinterpret_cast<float4 *>(prm.ws_o + ((size_t)split * rows + row_id) * D);
+        // The partial is written through shared memory so that global stores are
+        // whole rows: each warp stages its 32 rows, half of D at a time, in its
+        // own slice of this group's Q buffer (free once the group's last product
+        // has completed: every product of the group precedes its last PV), XOR-
+        // swizzled by row so that neither side of the transpose has bank conflicts.
+        constexpr int kScrCols = D / 2;
+        constexpr int kChunks = kScrCols / 4;                   // 16-byte chunks per staged row
+        constexpr int kRowsPerStore = 32 / kChunks;
+        float4 *scr = reinterpret_cast<float4 *>(sQ + grp * L::kQGroupBytes + sub * (32 * kScrCols * 4));
+        const long long my_off = row_valid ? (long long)(((size_t)split * rows + row_id) * D) : -1ll;
         if (have_o) tc_fence_after();
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t rr[32];
-            if (have_o) {
-                tmem_ld_32x32b_x32(tO + lane_addr + c0, rr);     // warp-collective: all lanes
-                tmem_ld_wait();
-            } else {
+        for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) rr[x] = 0u;
-            }
-            if (row_valid) {
+            for (int c0 = 0; c0 < kScrCols; c0 += 32) {
+                uint32_t rr[32];
+                if (have_o) {
+                    tmem_ld_32x32b_x32(tO + lane_addr + pass * kScrCols + c0, rr);   // warp-collective
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) rr[x] = 0u;
+                }
 #pragma unroll
                 for (int x = 0; x < 8; ++x)
-                    po[c0 / 4 + x] = make_float4(__uint_as_float(rr[4 * x]), __uint_as_float(rr[4 * x + 1]),
-                                                 __uint_as_float(rr[4 * x + 2]), __uint_as_float(rr[4 * x + 3]));
+                    scr[lane * kChunks + ((c0 / 4 + x) ^ (lane & (kChunks - 1)))] =
+                        make_float4(__uint_as_float(rr[4 * x]), __uint_as_float(rr[4 * x + 1]),
+                                    __uint_as_float(rr[4 * x + 2]), __uint_as_float(rr[4 * x + 3]));
             }
+            __syncwarp();
+#pragma unroll 4
+            for (int i = 0; i < 32; i += kRowsPerStore) {
+                const int wr = i + lane / kChunks, ch = lane % kChunks;
+                const long long off = __shfl_sync(0xffffffffu, my_off, wr);
+                const float4 v = scr[wr * kChunks + (ch ^ (wr & (kChunks - 1)))];
+                if (off >= 0) *reinterpret_cast<float4 *>(prm.ws_o + off + pass * kScrCols + ch * 4) = v;
+            }
+            __syncwarp();
         }
         if (row_valid) {
             prm.ws_ml[((size_t)split * rows + row_id) * 2 + 0] = m_used;
@@ -679,7 +764,13 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
     prm.ws_o = static_cast<float *>(ws);
     prm.ws_ml = prm.ws_o + (size_t)S * rows * D;
 
-    CUtensorMap tmK, tmV;
+    CUtensorMap tmK, tmV, tmQ;
+    memset(&tmQ, 0, sizeof(tmQ));
+    prm.q_tma = (kGroupRows % G == 0 &&
+                 encode_tensor_map_3d(&tmQ, q, D, a.Hq, a.total_nodes, (uint64_t)D * 2, (uint64_t)a.Hq * D * 2, 64,
+                                      G, kGroupRows / G))
+                    ? 1
+                    : 0;
     const uint64_t slots = (uint64_t)a.num_pages * a.page_size;
     if (!encode_tensor_map_3d(&tmK, k_cache, D, a.Hkv, slots, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2, 64, 1, 16))
         return cudaErrorInvalidValue;
@@ -696,7 +787,7 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
         attr_set[dev] = true;
     }
     dim3 grid((a.max_nodes * G + kRowsPerCta - 1) / kRowsPerCta, S, a.B * a.Hkv);
-    cudaError_t le = launch_pdl(tree_attention_tc_kernel<D>, grid, dim3(kAttnThreads), smem, st, tmK, tmV, prm);
+    cudaError_t le = launch_pdl(tree_attention_tc_kernel<D>, grid, dim3(kAttnThreads), smem, st, tmK, tmV, tmQ, prm);
     if (le != cudaSuccess) {
         cudaFuncAttributes fa;
         if (cudaFuncGetAttributes(&fa, tree_attention_tc_kernel<D>) == cudaSuccess)
