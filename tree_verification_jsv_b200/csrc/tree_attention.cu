@@ -64,6 +64,64 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction per pair).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rm.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^x for a pair on the FMA pipe, to take part of the exponentials off the
+// MUFU unit: x = j + f with j = floor(x) (from adding 1.5 * 2^23 rounded
+// toward -inf), 2^f on [0, 1) from a cubic with p(0) = 1 whose coefficients
+// are a minimax fit of the relative error (8.6e-5, well below the bf16
+// rounding of P), and j added into the exponent field.  Inputs below -127
+// are clamped there, where the result is exactly +0; inputs are at most 8.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    x = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+    const uint64_t t = f2_add_rm(x, magic);
+    const uint64_t f = f2_sub(x, f2_sub(t, magic));
+    uint64_t p = f2_fma(f2_pack(0.07706724f, 0.07706724f), f, f2_pack(0.22764498f, 0.22764498f));
+    p = f2_fma(p, f, f2_pack(0.69511663f, 0.69511663f));
+    p = f2_fma(p, f, f2_pack(1.f, 1.f));
+    float p0, p1, t0, t1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(t, t0, t1);
+    return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                   __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
 struct AttnParams {
     BatchArgs a;
     const uint16_t *q;
@@ -508,9 +566,9 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     tmem_st_wait();
                 }
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    mx[x & 3] = fmaxf(mx[x & 3], __uint_as_float(ra[x]));
-                    mx[x & 3] = fmaxf(mx[x & 3], __uint_as_float(rb[x]));
+                for (int x = 0; x < 32; x += 2) {
+                    mx[(x >> 1) & 3] = fmax3(mx[(x >> 1) & 3], __uint_as_float(ra[x]), __uint_as_float(ra[x + 1]));
+                    mx[(x >> 1) & 3] = fmax3(mx[(x >> 1) & 3], __uint_as_float(rb[x]), __uint_as_float(rb[x + 1]));
                 }
             }
             const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
@@ -543,30 +601,40 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 
             // pass 2: probabilities (masked columns hold -inf and give 0), their sum,
             // and the bf16 P row stored into the first 64 columns of this S buffer
+            // (pairs in packed fp32; one pair in four takes the polynomial 2^x)
             const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
-            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint64_t sl2x2 = f2_pack(sl2, sl2), negmx2 = f2_pack(neg_m, neg_m);
+            uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-            for (int c = 0; c < kKeyTile / 32; c += 2) {
-                uint32_t ra[32], rb[32];
+            for (int c = 0; c < kKeyTile / 32; ++c) {
+                uint32_t ra[32];
                 tmem_ld_32x32b_x32(sbase + c * 32, ra);
-                tmem_ld_32x32b_x32(sbase + (c + 1) * 32, rb);
                 tmem_ld_wait();
-                uint32_t pk[32];
+                uint32_t pk[16];
 #pragma unroll
                 for (int x = 0; x < 32; x += 2) {
-                    const float a0 = fast_exp2(fmaf(__uint_as_float(ra[x]), sl2, neg_m));
-                    const float a1 = fast_exp2(fmaf(__uint_as_float(ra[x + 1]), sl2, neg_m));
-                    const float b0 = fast_exp2(fmaf(__uint_as_float(rb[x]), sl2, neg_m));
-                    const float b1 = fast_exp2(fmaf(__uint_as_float(rb[x + 1]), sl2, neg_m));
-                    ps[(x >> 1) & 3] += (a0 + a1) + (b0 + b1);
+                    const uint64_t xa = f2_fma(f2_pack(__uint_as_float(ra[x]), __uint_as_float(ra[x + 1])), sl2x2, negmx2);
+                    uint64_t ea;
+                    if (((x >> 1) & 3) == 3) {
+                        ea = exp2_poly_x2(xa);
+                    } else {
+                        float u0, u1;
+                        f2_unpack(xa, u0, u1);
+                        ea = f2_pack(fast_exp2(u0), fast_exp2(u1));
+                    }
+                    ps2[(x >> 1) & 1] = f2_add(ps2[(x >> 1) & 1], ea);
+                    float a0, a1;
+                    f2_unpack(ea, a0, a1);
                     pk[x / 2] = pack_bf16x2(a0, a1);
-                    pk[16 + x / 2] = pack_bf16x2(b0, b1);
                 }
-                // keys [32c, 32c + 64) -> packed columns [16c, 16c + 32): columns the
+                // keys [32c, 32c + 32) -> packed columns [16c, 16c + 16): columns the
                 // loads above have already consumed
-                tmem_st_32x32b_x32(sbase + c * 16, pk);
+                tmem_st_32x32b_x16(sbase + c * 16, pk);
             }
-            const float psum = (ps[0] + ps[1]) + (ps[2] + ps[3]);
+            float q0, q1, q2, q3;
+            f2_unpack(ps2[0], q0, q1);
+            f2_unpack(ps2[1], q2, q3);
+            const float psum = (q0 + q1) + (q2 + q3);
             l = l * corr + psum;
             m_used = m_new;
             tmem_st_wait();
