@@ -16,18 +16,21 @@
 // partial (O, row max, row sum); a small combine kernel merges the splits
 // with log-sum-exp rescaling and rounds to bf16.
 //
-// Per CTA, 10 warps:
-//   warp 0      TMA producer: K and V of each 128-key tile, one 16-slot
-//               page x 64-dim box per copy, into a 2-stage ring; the warp
-//               looks up the next tile's pages while it waits for a stage
+// Per CTA, 12 warps (three warpgroups):
+//   warp 0      TMA producer: Q once, then K and V of each 128-key tile, one
+//               16-slot page x 64-dim box per copy, into a 2-stage ring; the
+//               warp looks up the next tile's pages while it waits for a stage
 //   warp 1      TMEM allocator and single-thread MMA issuer, in the order
 //               S0_0 S1_0 | PV0_0 S0_1 PV1_0 S1_1 | PV0_1 S0_2 ...
 //               (Sg_j = Q_g K_j^T, PVg_j: O_g += P_g V_j with P read from TMEM)
-//   warps 2..5  softmax of row group 0, warps 6..9 of row group 1: one query
-//               row per thread; masked online softmax in the log2 domain;
-//               P_j (bf16) is written over its own S buffer in TMEM; O is
-//               rescaled in TMEM only when the running max grows by more
-//               than 8 (2^8), which keeps exp2 arguments bounded
+//   warps 2, 3  idle (they complete the first warpgroup, which hands most of
+//               its registers to the other two)
+//   warps 4..7  softmax of row group 0, warps 8..11 of row group 1: one query
+//               row per thread, the whole 128-column row of S read from TMEM
+//               into registers at once; masked online softmax in the log2
+//               domain; P_j (bf16) is written over its own S buffer in TMEM;
+//               O is rescaled in TMEM only when the running max grows by
+//               more than 8 (2^8), which keeps exp2 arguments bounded
 // While one group computes its softmax the tensor core runs the other
 // group's products, so neither the exp2 pipe nor the tensor pipe waits on
 // the other for long.
@@ -47,7 +50,13 @@ using namespace sm100;
 constexpr int kGroups = 2;
 constexpr int kGroupRows = 128;
 constexpr int kRowsPerCta = kGroups * kGroupRows;
-constexpr int kAttnThreads = 64 + kGroups * 128;
+constexpr int kSoftmaxWarp0 = 4;              // warps 0..3: producer, MMA, two idle
+constexpr int kAttnThreads = 32 * kSoftmaxWarp0 + kGroups * 128;
+// registers a thread after the split (launch: 168 for all 12 warps); the
+// three warps of an SMSP hold 56 + 224 + 224 of its 512 registers a lane, and
+// 128 x 56 + 256 x 224 equals the 384 x 168 the CTA is launched with
+constexpr int kRegsControl = 56;
+constexpr int kRegsSoftmax = 224;
 constexpr int kKeyTile = 128;
 constexpr int kStages = 2;
 constexpr int kMaxTreeWords = 16;          // 512 nodes
@@ -222,6 +231,8 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         return j < (t_end - t_begin) ? (t_begin + j) * kKeyTile : P0 + (j - (t_end - t_begin)) * kKeyTile;
     };
 
+    if (warp < kSoftmaxWarp0) {
+    setmaxnreg_dec<kRegsControl>();
     if (warp == 0) {
         // ----------------------------------------------------------- producer
         // The whole warp runs the loop: lanes 0..7 look up the 8 physical pages
@@ -407,16 +418,18 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             mma_commit(&drain_bar);
             mbar_wait(&drain_bar, 0, (volatile int *)&zero);
         }
+    }
     } else {
+        setmaxnreg_inc<kRegsSoftmax>();
         // ----------------------------------------------------------- softmax
-        const int grp = (warp - 2) >> 2;             // row group of this warp
+        const int grp = (warp - kSoftmaxWarp0) >> 2;  // row group of this warp
         const int sub = warp & 3;                    // TMEM lanes this warp may access
         const int grow = sub * 32 + lane;            // row within the group == TMEM lane
         const int row = grp * kGroupRows + grow;     // row within the CTA tile
         const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
         const uint32_t tS = tmem + grp * 128;
         const uint32_t tO = tmem + 256 + grp * D;
-        const int et = threadIdx.x - 64;             // 0..255
+        const int et = threadIdx.x - 32 * kSoftmaxWarp0;   // 0..255
         const bool row_valid = row < rows_here;
         const int rg = m0 + row;                     // row within (b, g)
         const int node = rg / G;                     // request-local node
@@ -502,7 +515,6 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         float m_used = -INFINITY, l = 0.f;
         const float sl2 = prm.scale_log2;
         bool ok = true;
-        int o_seen = 0;                              // PV completions observed
         const int my_tiles = grp < ngroups ? ntiles : 0;
         for (int j = 0; j < my_tiles; ++j) {
             if (!mbar_wait(&s_full[grp], j & 1, &abort_sh)) ok = false;
@@ -511,64 +523,49 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             const int slot0 = tile_slot0(j);
             const bool is_tree = j >= (t_end - t_begin);
             const uint32_t sbase = tS + lane_addr;
-            // one visibility word per 32-key chunk: bit x <-> key column c0 + x
-            uint32_t vis[kKeyTile / 32];
+            // The whole 128-column row of S in registers: one TMEM round trip.
+            uint32_t sv[kKeyTile / 32][32];
 #pragma unroll
-            for (int c = 0; c < kKeyTile / 32; ++c) {
-                const int s0 = slot0 + c * 32;
-                if (!is_tree) {
-                    const int cnt = r.P - s0;
-                    vis[c] = cnt >= 32 ? 0xffffffffu : (cnt <= 0 ? 0u : ((1u << cnt) - 1u));
-                } else {
-                    const int j0 = s0 - r.P;             // tree node of column c*32 (may be < 0)
-                    uint32_t wv = 0u;
-                    if (row_valid && j0 > -32 && j0 < 32 * kMaxTreeWords) {
-                        if (j0 < 0) {
-                            wv = anc[row][0] << (-j0);
-                        } else {
-                            const int w = j0 >> 5;
-                            const uint32_t lo = anc[row][w];
-                            const uint32_t hi = (w + 1 < kMaxTreeWords) ? anc[row][w + 1] : 0u;
-                            wv = __funnelshift_r(lo, hi, j0 & 31);
+            for (int c = 0; c < kKeyTile / 32; ++c) tmem_ld_32x32b_x32(sbase + c * 32, sv[c]);
+            tmem_ld_wait();
+            // Masked columns (past the prefix in its last tile; non-ancestors in
+            // tree tiles) become -inf.  One visibility word per 32-key chunk:
+            // bit x <-> key column 32c + x.
+            if (slot0 + kKeyTile > r.P) {
+#pragma unroll
+                for (int c = 0; c < kKeyTile / 32; ++c) {
+                    const int s0 = slot0 + c * 32;
+                    uint32_t vis;
+                    if (!is_tree) {
+                        const int cnt = r.P - s0;
+                        vis = cnt >= 32 ? 0xffffffffu : (cnt <= 0 ? 0u : ((1u << cnt) - 1u));
+                    } else {
+                        const int j0 = s0 - r.P;         // tree node of column 32c (may be < 0)
+                        vis = 0u;
+                        if (row_valid && j0 > -32 && j0 < 32 * kMaxTreeWords) {
+                            if (j0 < 0) {
+                                vis = anc[row][0] << (-j0);
+                            } else {
+                                const int w = j0 >> 5;
+                                const uint32_t lo = anc[row][w];
+                                const uint32_t hi = (w + 1 < kMaxTreeWords) ? anc[row][w + 1] : 0u;
+                                vis = __funnelshift_r(lo, hi, j0 & 31);
+                            }
                         }
                     }
-                    vis[c] = wv;
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) sv[c][x] = ((vis >> x) & 1u) ? sv[c][x] : 0xff800000u;
                 }
             }
-            // pass 1: row max of the raw scores (the scale is positive).  Chunks with
-            // masked columns get -inf written back into TMEM, so pass 2 needs no mask.
+            // row max of the raw scores (the scale is positive)
             float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < kKeyTile / 32; c += 2) {
-                uint32_t ra[32], rb[32];
-                tmem_ld_32x32b_x32(sbase + c * 32, ra);
-                tmem_ld_32x32b_x32(sbase + (c + 1) * 32, rb);
-                tmem_ld_wait();
-                if (__any_sync(0xffffffffu, (vis[c] & vis[c + 1]) != 0xffffffffu)) {
+            for (int c = 0; c < kKeyTile / 32; ++c) {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        ra[x] = ((vis[c] >> x) & 1u) ? ra[x] : 0xff800000u;
-                        rb[x] = ((vis[c + 1] >> x) & 1u) ? rb[x] : 0xff800000u;
-                    }
-                    uint32_t h[16];
+                for (int x = 0; x < 32; x += 8) {
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) h[x] = ra[x];
-                    tmem_st_32x32b_x16(sbase + c * 32, h);
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) h[x] = ra[16 + x];
-                    tmem_st_32x32b_x16(sbase + c * 32 + 16, h);
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) h[x] = rb[x];
-                    tmem_st_32x32b_x16(sbase + (c + 1) * 32, h);
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) h[x] = rb[16 + x];
-                    tmem_st_32x32b_x16(sbase + (c + 1) * 32 + 16, h);
-                    tmem_st_wait();
-                }
-#pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                    mx[(x >> 1) & 3] = fmax3(mx[(x >> 1) & 3], __uint_as_float(ra[x]), __uint_as_float(ra[x + 1]));
-                    mx[(x >> 1) & 3] = fmax3(mx[(x >> 1) & 3], __uint_as_float(rb[x]), __uint_as_float(rb[x + 1]));
+                    for (int u = 0; u < 4; ++u)
+                        mx[u] = fmax3(mx[u], __uint_as_float(sv[c][x + 2 * u]), __uint_as_float(sv[c][x + 2 * u + 1]));
                 }
             }
             const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
@@ -577,16 +574,10 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             if (tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY)) m_new = tmax;
             const float corr = (m_new == m_used) ? 1.f : fast_exp2(m_used - m_new);   // 0 when m_used = -inf
 
-            // O holds P_0..P_{j-1} V under the old max: rescale it (rarely) once
-            // PV_{j-1} has completed.  o_seen counts the PV completions observed;
-            // they are observed one by one, so the parity wait never aliases.
+            // O holds P_0..P_{j-1} V under the old max: rescale it (rarely).  S_j
+            // was issued after PV_{j-1} and its completion covers every earlier
+            // product of the issuing thread, so PV_{j-1} is complete here.
             if (__any_sync(0xffffffffu, corr != 1.f) && j >= 1) {
-                while (o_seen <= j - 1) {
-                    if (!mbar_wait(&o_done[grp], o_seen & 1, &abort_sh)) ok = false;
-                    ++o_seen;
-                }
-                if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-                tc_fence_after();
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t ov[32];
@@ -599,38 +590,32 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 tmem_st_wait();
             }
 
-            // pass 2: probabilities (masked columns hold -inf and give 0), their sum,
-            // and the bf16 P row stored into the first 64 columns of this S buffer
-            // (pairs in packed fp32; one pair in four takes the polynomial 2^x)
+            // probabilities (masked columns hold -inf and give 0), their sum, and
+            // the bf16 P row stored into the first 64 columns of this S buffer;
+            // pairs in packed fp32, one pair in four through the polynomial 2^x
             const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
             const uint64_t sl2x2 = f2_pack(sl2, sl2), negmx2 = f2_pack(neg_m, neg_m);
             uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+            uint32_t pk[2][32];
 #pragma unroll
-            for (int c = 0; c < kKeyTile / 32; ++c) {
-                uint32_t ra[32];
-                tmem_ld_32x32b_x32(sbase + c * 32, ra);
-                tmem_ld_wait();
-                uint32_t pk[16];
-#pragma unroll
-                for (int x = 0; x < 32; x += 2) {
-                    const uint64_t xa = f2_fma(f2_pack(__uint_as_float(ra[x]), __uint_as_float(ra[x + 1])), sl2x2, negmx2);
-                    uint64_t ea;
-                    if (((x >> 1) & 3) == 3) {
-                        ea = exp2_poly_x2(xa);
-                    } else {
-                        float u0, u1;
-                        f2_unpack(xa, u0, u1);
-                        ea = f2_pack(fast_exp2(u0), fast_exp2(u1));
-                    }
-                    ps2[(x >> 1) & 1] = f2_add(ps2[(x >> 1) & 1], ea);
-                    float a0, a1;
-                    f2_unpack(ea, a0, a1);
-                    pk[x / 2] = pack_bf16x2(a0, a1);
+            for (int i = 0; i < kKeyTile / 2; ++i) {
+                const int c = (2 * i) / 32, x = (2 * i) % 32;
+                const uint64_t xa = f2_fma(f2_pack(__uint_as_float(sv[c][x]), __uint_as_float(sv[c][x + 1])), sl2x2, negmx2);
+                uint64_t ea;
+                if ((i & 3) == 3) {
+                    ea = exp2_poly_x2(xa);
+                } else {
+                    float u0, u1;
+                    f2_unpack(xa, u0, u1);
+                    ea = f2_pack(fast_exp2(u0), fast_exp2(u1));
                 }
-                // keys [32c, 32c + 32) -> packed columns [16c, 16c + 16): columns the
-                // loads above have already consumed
-                tmem_st_32x32b_x16(sbase + c * 16, pk);
+                ps2[i & 1] = f2_add(ps2[i & 1], ea);
+                float a0, a1;
+                f2_unpack(ea, a0, a1);
+                pk[i / 32][i % 32] = pack_bf16x2(a0, a1);
             }
+            tmem_st_32x32b_x32(sbase, pk[0]);
+            tmem_st_32x32b_x32(sbase + 32, pk[1]);
             float q0, q1, q2, q3;
             f2_unpack(ps2[0], q0, q1);
             f2_unpack(ps2[1], q2, q3);
@@ -638,12 +623,6 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             l = l * corr + psum;
             m_used = m_new;
             tmem_st_wait();
-            // observe PV_{j-1} before handing over P_j (PV_j cannot start before that)
-            while (o_seen <= j - 1) {
-                if (!mbar_wait(&o_done[grp], o_seen & 1, &abort_sh)) ok = false;
-                ++o_seen;
-            }
-            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[grp]);
@@ -652,10 +631,10 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         // final partial: O (unnormalised), running max (log2 domain) and sum
         bool have_o = ok && my_tiles > 0;
         if (have_o) {
-            while (o_seen <= my_tiles - 1) {
-                if (!mbar_wait(&o_done[grp], o_seen & 1, &abort_sh)) ok = false;
-                ++o_seen;
-            }
+            // the last PV: every earlier one is complete (the last S came after
+            // it), so the barrier is in phase my_tiles - 1 or past it and this
+            // parity wait cannot alias
+            if (!mbar_wait(&o_done[grp], (uint32_t)((my_tiles - 1) & 1), &abort_sh)) ok = false;
             if (__any_sync(0xffffffffu, !ok)) have_o = false;
         }
         if (!have_o) {
