@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import attention_close, bf16, small_case
+from helpers import attention_close, bf16, dense_tree_attention, small_case
 from tree_verification_jsv_b200 import jsv, synth
 
 pytestmark = pytest.mark.gpu
@@ -205,3 +205,15 @@ def test_page_out_of_range_is_reported():
     case["page_table"][0, 1] = case["num_pages"] + 5
     out, st = run_attention(case)
     assert st == jsv.JSV_ERR_DEVICE_INPUT
+
+
+# Chains whose row counts straddle the 64-, 128- and 256-row boundaries of the
+# CTA's row groups and warps, with one and several key tiles: each warp of a
+# group may run a tile ahead of the others, and every row must still see the
+# P of its own tile.
+@pytest.mark.parametrize("n,pre", [(30, 29), (33, 29), (41, 29), (64, 29), (64, 200), (41, 300)])
+def test_attention_row_groups_and_tiles(n, pre):
+    case = small_case([np.arange(-1, n - 1)], [pre], Hq=8, Hkv=2, D=128, seed=11)
+    got, st = run_attention(case)
+    assert st == 0
+    attention_close(got, dense_tree_attention(case), f"chain n={n} prefix={pre}")

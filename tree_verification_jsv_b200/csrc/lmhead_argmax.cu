@@ -7,23 +7,25 @@
 //
 // Shape of the contraction: logits^T[v][t] = W[v][:] . H[t][:].  The
 // vocabulary is the MMA M dimension (128 rows per tile, operand A = W) and
-// the tree nodes are the N dimension (operand B = H), so a 64-node tree
-// still fills M = 128 and W -- the dominant byte stream -- is read exactly
-// once when T <= 512.
+// the tree nodes are the N dimension (operand B = H, up to 256 nodes per
+// MMA), so a 64-node tree still fills M = 128.
 //
+// An item is one 128-row vocabulary tile x one group of up to 256 nodes.
 // Persistent kernel, one CTA per SM, 6 warps:
-//   warp 0      TMA producer: W tile (16-row boxes) + H tile per 64-wide K
-//               chunk into a ring of shared-memory stages
+//   warp 0      TMA producer: W tile (16-row boxes for a ragged tile) + H
+//               tile per 64-wide K chunk into a ring of shared-memory stages
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator, per-column argmax
 //               across the 128 vocabulary rows (a transposing butterfly of
 //               64-bit keys), then one atomicMax per node
-// Each CTA owns a contiguous, balanced vocabulary range [V*c/G, V*(c+1)/G)
-// and walks it in 128-row tiles; the ragged last tile of a range loads only
-// the 16-row boxes it needs, so no SM gets a whole extra tile of bytes.
-// With T <= 256 nodes two accumulators alternate in TMEM so the epilogue of
-// one tile overlaps the main loop of the next; larger trees are processed in
-// groups of 512 nodes (two N = 256 MMAs per K step, one accumulator).
+// Two accumulators alternate in TMEM, so the epilogue of one item overlaps
+// the main loop of the next.
+// Work split: with one node group (up to 256 nodes; W, the dominant byte
+// stream, is read exactly once) each CTA owns a contiguous, balanced
+// vocabulary range [V*c/G, V*(c+1)/G) whose ragged last tile loads only the
+// 16-row boxes it needs.  With several node groups the tensor pipe
+// dominates: each CTA takes a balanced contiguous range of the (tile, group)
+// items, group fastest, so consecutive items reuse the same W tile from L2.
 //
 // Cross-CTA reduction: a 64-bit key per node whose high word is the fp32
 // value mapped to an order-preserving unsigned integer and whose low word is
@@ -56,32 +58,20 @@ __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsig
 
 
 constexpr int kMaxStages = 8;
-constexpr int kTileM = 128;                    // MMA M (one sub-tile)
+constexpr int kTileM = 128;                    // MMA M: vocabulary rows of a tile
+constexpr int kMaxGroupNodes = 256;            // MMA N: nodes of a group
 constexpr int kBoxRowsW = 16;
 constexpr int kKChunk = 64;                    // bf16 elements per 128-B swizzle line
-constexpr uint32_t kSubA = kTileM * 128;       // 16 KB: one sub-tile's K-chunk
+constexpr uint32_t kStageA = kTileM * 128;     // 16 KB: a W tile's K-chunk
 constexpr int kSmemBudget = 200 * 1024;        // ring of stages (dynamic smem)
-
-// An item is kSub 128-row vocabulary sub-tiles x one node group; the sub-tiles
-// share each K-chunk of the node tile.  One sub-tile suits trees of up to 256
-// nodes (W streaming dominates); two halve the node-tile traffic for larger
-// trees, where the tensor pipe dominates.
-template <int kSub>
-struct LmShape {
-    static constexpr int kEpiWarps = 4 * kSub;     // kSub epilogue warps per TMEM subpartition
-    static constexpr int kThreads = 64 + 32 * kEpiWarps;
-    static constexpr int kItemRows = kTileM * kSub;
-    static constexpr uint32_t kStageA = kSubA * kSub;
-};
+constexpr int kEpiWarps = 4;                   // one per TMEM subpartition
+constexpr int kLmThreads = 64 + 32 * kEpiWarps;
 
 struct LmParams {
     int T, d, V;
     int kchunks;       // d / 64
     int ngroups;       // node groups
-    int group_nodes;   // nodes per group (<= 256)
-    int box_rows;      // H box height (= MMA N of a full group)
-    int sub_stride;    // TMEM columns between the two sub-tile accumulators
-    int n_acc;         // accumulator sets in TMEM (2 = double buffered, 1)
+    int group_nodes;   // nodes per group (<= 256): the H box height
     int stages;
     uint32_t stage_bytes;
     unsigned long long *keys;
@@ -91,34 +81,67 @@ struct LmParams {
     int32_t *status;
 };
 
+// The k-th item of a CTA: vocabulary rows [row0, row0 + rows) and node group g.
+struct LmItem {
+    int row0, rows, g;
+};
+
+struct LmWork {
+    int r0, r1;        // vocabulary range (one node group)
+    int it0;           // first global item (several node groups)
+    int items;
+
+    __device__ LmWork(const LmParams &p, int cta, int G) {
+        if (p.ngroups == 1) {
+            r0 = (int)((long long)p.V * cta / G);
+            r1 = (int)((long long)p.V * (cta + 1) / G);
+            it0 = 0;
+            items = (r1 - r0 + kTileM - 1) / kTileM;
+        } else {
+            const long long total = (long long)((p.V + kTileM - 1) / kTileM) * p.ngroups;
+            r0 = r1 = 0;
+            it0 = (int)(total * cta / G);
+            items = (int)(total * (cta + 1) / G) - it0;
+        }
+    }
+    __device__ LmItem item(const LmParams &p, int k) const {
+        LmItem t;
+        if (p.ngroups == 1) {
+            t.row0 = r0 + k * kTileM;
+            t.rows = min(kTileM, r1 - t.row0);
+            t.g = 0;
+        } else {
+            const int i = it0 + k, vt = i / p.ngroups;
+            t.row0 = vt * kTileM;
+            t.rows = min(kTileM, p.V - t.row0);
+            t.g = i - vt * p.ngroups;
+        }
+        return t;
+    }
+};
+
 __device__ __forceinline__ void set_abort(volatile int *abort, int32_t *status) {
     *abort = 1;
     if (status) atomicCAS(status, 0, JSV_ERR_TIMEOUT);
 }
 
-template <int kSubTiles>
-__global__ void __launch_bounds__(LmShape<kSubTiles>::kThreads, 1)
+__global__ void __launch_bounds__(kLmThreads, 1)
 lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmW16,
                         const __grid_constant__ CUtensorMap tmH, const LmParams p) {
     pdl_allow_dependents();
     pdl_wait_predecessor();
-    constexpr int kEpiWarps = LmShape<kSubTiles>::kEpiWarps;
-    constexpr int kItemRows = LmShape<kSubTiles>::kItemRows;
-    constexpr uint32_t kStageA = LmShape<kSubTiles>::kStageA;
     extern __shared__ uint8_t dsmem[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
     __shared__ __align__(8) uint64_t accf_bar[2], acce_bar[2], drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ volatile int ep_fail;
-    __shared__ unsigned long long red[kEpiWarps][256];
+    __shared__ unsigned long long red[kEpiWarps][kMaxGroupNodes];
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = gridDim.x, cta = blockIdx.x;
-    const int r0 = (int)((long long)p.V * cta / G), r1 = (int)((long long)p.V * (cta + 1) / G);
-    const int ntiles = (r1 - r0 + kItemRows - 1) / kItemRows;
-    const int items = ntiles * p.ngroups;
+    const LmWork work(p, blockIdx.x, gridDim.x);
+    const int items = work.items;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -151,22 +174,19 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();
+            // W is read once with one node group (stream it past L2), several
+            // times from L2 with several; H is re-read by every item
+            const uint64_t pol_w = p.ngroups == 1 ? policy_evict_first() : policy_evict_normal();
             const uint64_t pol_h = policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
             for (int it = 0; it < items && !abort_sh; ++it) {
-                const int vt = it / p.ngroups, g = it % p.ngroups;
-                const int row0 = r0 + vt * kItemRows;
-                int rows[kSubTiles];
-                uint32_t tx = (uint32_t)p.box_rows * 128;
-#pragma unroll
-                for (int s = 0; s < kSubTiles; ++s) {
-                    rows[s] = max(0, min(kTileM, r1 - (row0 + s * kTileM)));
-                    tx += rows[s] == kTileM ? kSubA : (uint32_t)((rows[s] + kBoxRowsW - 1) / kBoxRowsW) * (kBoxRowsW * 128);
-                }
-                const int node0 = g * p.group_nodes;
+                const LmItem t = work.item(p, it);
+                const uint32_t tx = (uint32_t)p.group_nodes * 128 +
+                                    (t.rows == kTileM ? kStageA
+                                                      : (uint32_t)((t.rows + kBoxRowsW - 1) / kBoxRowsW) * (kBoxRowsW * 128));
+                const int node0 = t.g * p.group_nodes;
                 bool ok = true;
                 for (int kc = 0; kc < p.kchunks; ++kc) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh)) {
@@ -177,16 +197,12 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
                     uint8_t *sa = smem + (size_t)stage * p.stage_bytes;
                     uint8_t *sb = sa + kStageA;
                     mbar_arrive_expect_tx(&full_bar[stage], tx);
-#pragma unroll
-                    for (int s = 0; s < kSubTiles; ++s) {
-                        const int rs = row0 + s * kTileM;
-                        if (rows[s] == kTileM) {
-                            tma_load_2d_hint(sa + s * kSubA, &tmW, &full_bar[stage], kc * kKChunk, rs, pol_w);
-                        } else {
-                            for (int bx = 0; bx * kBoxRowsW < rows[s]; ++bx)
-                                tma_load_2d_hint(sa + s * kSubA + bx * (kBoxRowsW * 128), &tmW16, &full_bar[stage],
-                                                 kc * kKChunk, rs + bx * kBoxRowsW, pol_w);
-                        }
+                    if (t.rows == kTileM) {
+                        tma_load_2d_hint(sa, &tmW, &full_bar[stage], kc * kKChunk, t.row0, pol_w);
+                    } else {
+                        for (int bx = 0; bx * kBoxRowsW < t.rows; ++bx)
+                            tma_load_2d_hint(sa + bx * (kBoxRowsW * 128), &tmW16, &full_bar[stage], kc * kKChunk,
+                                             t.row0 + bx * kBoxRowsW, pol_w);
                     }
                     tma_load_2d_hint(sb, &tmH, &full_bar[stage], kc * kKChunk, node0, pol_h);
                     ++issued;
@@ -213,17 +229,15 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
             int stage = 0;
             uint32_t phase = 0;
             for (int it = 0; it < items && !abort_sh; ++it) {
-                const int acc = it % p.n_acc;
-                const uint32_t use = (uint32_t)(it / p.n_acc);
+                const int acc = it & 1;
+                const uint32_t use = (uint32_t)(it >> 1);
                 if (!mbar_wait(&acce_bar[acc], (use & 1) ^ 1, &abort_sh)) {
                     set_abort(&abort_sh, p.status);
                     break;
                 }
                 tc_fence_after();
-                const int vt = it / p.ngroups, g = it % p.ngroups;
-                const int row0 = r0 + vt * kItemRows;
-                const bool sub1 = kSubTiles > 1 && r1 - (row0 + kTileM) > 0;   // second sub-tile has rows
-                const int in_group = min(p.group_nodes, p.T - g * p.group_nodes);
+                const LmItem t = work.item(p, it);
+                const int in_group = min(p.group_nodes, p.T - t.g * p.group_nodes);
                 const uint32_t idn = idesc_bf16_f32(kTileM, (in_group + 15) & ~15, false, false);
                 const uint32_t d0 = tmem + (uint32_t)acc * 256u;
                 bool ok = true;
@@ -237,14 +251,9 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
                     const uint32_t sa = smem_addr(smem + (size_t)stage * p.stage_bytes);
                     const uint32_t sb = sa + kStageA;
 #pragma unroll
-                    for (int kk = 0; kk < kKChunk / 16; ++kk) {
-                        const uint32_t accum = (kc | kk) != 0;
-                        const uint64_t bdesc = desc_kmajor_sw128(sb + kk * 32);
-                        mma_bf16_ss(d0, desc_kmajor_sw128(sa + kk * 32), bdesc, idn, accum);
-                        if (kSubTiles > 1 && sub1)
-                            mma_bf16_ss(d0 + (uint32_t)p.sub_stride, desc_kmajor_sw128(sa + kSubA + kk * 32), bdesc,
-                                        idn, accum);
-                    }
+                    for (int kk = 0; kk < kKChunk / 16; ++kk)
+                        mma_bf16_ss(d0, desc_kmajor_sw128(sa + kk * 32), desc_kmajor_sw128(sb + kk * 32), idn,
+                                    (kc | kk) != 0);
                     mma_commit(&empty_bar[stage]);
                     if (++stage == p.stages) { stage = 0; phase ^= 1; }
                 }
@@ -258,14 +267,13 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int ew = warp - 2;                     // 0..7
-        const int subt = ew >> 2;                    // vocabulary sub-tile this warp reads
+        const int ew = warp - 2;                     // 0..3
         const int sub = warp & 3;                    // TMEM lanes this warp may access
         const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
-        const int et = threadIdx.x - 64;             // 0..255
+        const int et = threadIdx.x - 64;             // 0..127
         for (int it = 0; it < items; ++it) {
-            const int acc = it % p.n_acc;
-            const uint32_t use = (uint32_t)(it / p.n_acc);
+            const int acc = it & 1;
+            const uint32_t use = (uint32_t)(it >> 1);
             if (!mbar_wait(&accf_bar[acc], use & 1, &abort_sh)) {
                 set_abort(&abort_sh, p.status);
                 ep_fail = 1;
@@ -273,13 +281,13 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
             named_barrier(1, 32 * kEpiWarps);
             if (ep_fail) break;
             tc_fence_after();
-            const int vt = it / p.ngroups, g = it % p.ngroups;
-            const int v = r0 + vt * kItemRows + subt * kTileM + sub * 32 + lane;
-            const bool vvalid = v < r1;
-            const int node0 = g * p.group_nodes;
+            const LmItem t = work.item(p, it);
+            const int v = t.row0 + sub * 32 + lane;
+            const bool vvalid = v < t.row0 + t.rows;
+            const int node0 = t.g * p.group_nodes;
             const int in_group = min(p.group_nodes, p.T - node0);
             const int ncols = (in_group + 31) & ~31;
-            const uint32_t base = tmem + lane_addr + (uint32_t)acc * 256u + (uint32_t)(subt * p.sub_stride);
+            const uint32_t base = tmem + lane_addr + (uint32_t)acc * 256u;
             for (int c0 = 0; c0 < ncols; c0 += 32) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(base + (uint32_t)c0, r);
@@ -345,24 +353,12 @@ cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int 
                                  int32_t *argmax, float *max_logit, void *ws, cudaStream_t st) {
     int32_t *status = nullptr;
     auto *keys = static_cast<unsigned long long *>(ws);
-    const int sub = T <= 256 ? 1 : 2;
     LmParams p;
     p.T = T; p.d = d; p.V = V;
     p.kchunks = d / kKChunk;
-    if (sub == 1) {
-        // one 128-row accumulator per item, two items in flight in TMEM
-        p.group_nodes = (T + 15) & ~15;
-        p.sub_stride = 0;
-        p.n_acc = 2;
-    } else {
-        // two 128-row accumulators of up to 256 nodes fill TMEM: one item in flight
-        p.group_nodes = 256;
-        p.sub_stride = 256;
-        p.n_acc = 1;
-    }
-    p.box_rows = p.group_nodes;
+    p.group_nodes = min(kMaxGroupNodes, (T + 15) & ~15);
     p.ngroups = (T + p.group_nodes - 1) / p.group_nodes;
-    p.stage_bytes = kSubA * sub + (uint32_t)p.box_rows * 128;
+    p.stage_bytes = kStageA + (uint32_t)p.group_nodes * 128;
     p.stages = kSmemBudget / (int)p.stage_bytes;
     if (p.stages > kMaxStages) p.stages = kMaxStages;
     p.keys = keys;
@@ -376,32 +372,26 @@ cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int 
         return cudaErrorInvalidValue;
     if (!encode_tensor_map_2d(&tmW16, w, (uint64_t)d, (uint64_t)V, (uint64_t)d * 2, kKChunk, kBoxRowsW))
         return cudaErrorInvalidValue;
-    if (!encode_tensor_map_2d(&tmH, hidden, (uint64_t)d, (uint64_t)T, (uint64_t)d * 2, kKChunk, p.box_rows))
+    if (!encode_tensor_map_2d(&tmH, hidden, (uint64_t)d, (uint64_t)T, (uint64_t)d * 2, kKChunk, p.group_nodes))
         return cudaErrorInvalidValue;
 
     const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
-    static bool attr_set[64][2] = {};
+    static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev][sub - 1]) {
-        cudaError_t e = sub == 1 ? cudaFuncSetAttribute(lmhead_argmax_tc_kernel<1>,
-                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget + 1024)
-                                 : cudaFuncSetAttribute(lmhead_argmax_tc_kernel<2>,
-                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget + 1024);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(lmhead_argmax_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmemBudget + 1024);
         if (e != cudaSuccess) return e;
-        attr_set[dev][sub - 1] = true;
+        attr_set[dev] = true;
     }
     cudaError_t e = cudaMemsetAsync(keys, 0, lmhead_workspace_bytes(T, d, V), st);
     if (e != cudaSuccess) return e;
-    const int item_rows = kTileM * sub;
-    const int tiles = (V + item_rows - 1) / item_rows;
+    const long long items = (long long)((V + kTileM - 1) / kTileM) * p.ngroups;
     int grid = device_sm_count();
     if (grid <= 0) return cudaErrorInvalidDevice;
-    if (grid > tiles) grid = tiles;
-    if (sub == 1)
-        e = launch_pdl(lmhead_argmax_tc_kernel<1>, dim3(grid), dim3(LmShape<1>::kThreads), smem, st, tmW, tmW16, tmH, p);
-    else
-        e = launch_pdl(lmhead_argmax_tc_kernel<2>, dim3(grid), dim3(LmShape<2>::kThreads), smem, st, tmW, tmW16, tmH, p);
+    if (grid > items) grid = (int)items;
+    e = launch_pdl(lmhead_argmax_tc_kernel, dim3(grid), dim3(kLmThreads), smem, st, tmW, tmW16, tmH, p);
     count_launches(1);
     return e;
 }
