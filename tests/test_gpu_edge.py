@@ -93,7 +93,7 @@ def test_attention_edge_cases(name, sharp):
 
 
 @pytest.mark.parametrize("T,d,V", [(1, 64, 1), (5, 128, 1000), (16, 256, 1024), (64, 512, 4099),
-                                   (130, 192, 3000), (300, 1024, 20000)])
+                                   (130, 192, 3000), (300, 1024, 20000), (200, 256, 2500), (256, 128, 257)])
 def test_lmhead_argmax_shapes(T, d, V):
     rng = np.random.default_rng(T * 7 + V)
     H = bf16(rng.standard_normal((T, d)) / math.sqrt(d))
