@@ -367,19 +367,22 @@ struct LmPairItem {
     int row0, rows, g;     // the pair's rows [row0, row0 + rows), node group
 };
 
+// Items of a pair.  One node group: a contiguous, balanced vocabulary range
+// (W is read once).  Several: items (tile, group), group fastest, dealt out
+// round-robin -- pair p takes items p, p + npairs, ... -- so at any moment
+// neighbouring pairs work on the same W tile for different node groups and
+// each tile comes from HBM once and from L2 for the other groups.
 struct LmPairWork {
-    int r0, r1, it0, items;
-    __device__ LmPairWork(const LmParams &p, int pair, int npairs) {
+    int r0, r1, pair, npairs, items;
+    __device__ LmPairWork(const LmParams &p, int pair_, int npairs_) : pair(pair_), npairs(npairs_) {
         if (p.ngroups == 1) {
             r0 = (int)((long long)p.V * pair / npairs);
             r1 = (int)((long long)p.V * (pair + 1) / npairs);
-            it0 = 0;
             items = (r1 - r0 + kPairRows - 1) / kPairRows;
         } else {
             const long long total = (long long)((p.V + kPairRows - 1) / kPairRows) * p.ngroups;
             r0 = r1 = 0;
-            it0 = (int)(total * pair / npairs);
-            items = (int)(total * (pair + 1) / npairs) - it0;
+            items = (int)((total - pair + npairs - 1) / npairs);
         }
     }
     __device__ LmPairItem item(const LmParams &p, int k) const {
@@ -389,10 +392,11 @@ struct LmPairWork {
             t.rows = min(kPairRows, r1 - t.row0);
             t.g = 0;
         } else {
-            const int i = it0 + k, vt = i / p.ngroups;
+            const long long i = pair + (long long)k * npairs;
+            const int vt = (int)(i / p.ngroups);
             t.row0 = vt * kPairRows;
             t.rows = min(kPairRows, p.V - t.row0);
-            t.g = i - vt * p.ngroups;
+            t.g = (int)(i - (long long)vt * p.ngroups);
         }
         return t;
     }
