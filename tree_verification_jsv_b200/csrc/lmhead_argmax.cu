@@ -514,14 +514,23 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0 && rank == 0) {
+        // The whole warp runs the issue loop with warp-uniform operands (one
+        // elected lane issues); lane 0 waits on the barriers and broadcasts.
+        if (rank == 0) {
+            auto wait1 = [&](uint64_t *bar, uint32_t parity) -> bool {
+                int w = 1;
+                if (lane == 0) w = mbar_wait(bar, parity, &abort_sh) ? 1 : 0;
+                return __shfl_sync(0xffffffffu, w, 0) != 0;
+            };
+            const uint64_t da0 = desc_kmajor_sw128(smem_addr(smem));
+            const uint64_t db0 = desc_kmajor_sw128(smem_addr(smem + kStageA));
             int stage = 0;
             uint32_t phase = 0;
-            for (int it = 0; it < items && !abort_sh; ++it) {
+            for (int it = 0; it < items; ++it) {
                 const int acc = it & 1;
                 const uint32_t use = (uint32_t)(it >> 1);
-                if (!mbar_wait(&acce_bar[acc], (use & 1) ^ 1, &abort_sh)) {
-                    set_abort(&abort_sh, p.status);
+                if (!wait1(&acce_bar[acc], (use & 1) ^ 1)) {
+                    if (lane == 0) set_abort(&abort_sh, p.status);
                     break;
                 }
                 tc_fence_after();
@@ -531,26 +540,25 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
                 const uint32_t d0 = tmem + (uint32_t)acc * 256u;
                 bool ok = true;
                 for (int kc = 0; kc < p.kchunks; ++kc) {
-                    if (!mbar_wait(&full_bar[stage], phase, &abort_sh)) {
-                        set_abort(&abort_sh, p.status);
+                    if (!wait1(&full_bar[stage], phase)) {
+                        if (lane == 0) set_abort(&abort_sh, p.status);
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = smem_addr(smem + (size_t)stage * p.stage_bytes);
-                    const uint32_t sb = sa + kStageA;
+                    const uint64_t soff = (uint64_t)((stage * p.stage_bytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < kKChunk / 16; ++kk)
-                        mma_bf16_ss_pair(d0, desc_kmajor_sw128(sa + kk * 32), desc_kmajor_sw128(sb + kk * 32), idn,
-                                         (kc | kk) != 0);
-                    mma_commit_pair(&empty_bar[stage], 0x3);
+                        mma_bf16_ss_pair_warp(d0, da0 + soff + (uint64_t)(kk * 2), db0 + soff + (uint64_t)(kk * 2),
+                                              idn, (kc | kk) != 0);
+                    mma_commit_pair_warp(&empty_bar[stage], 0x3);
                     if (++stage == p.stages) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                mma_commit_pair(&accf_bar[acc], 0x3);
+                mma_commit_pair_warp(&accf_bar[acc], 0x3);
             }
             // every MMA issued above has finished before either CTA frees TMEM
-            mma_commit_pair(&drain_bar, 0x3);
+            mma_commit_pair_warp(&drain_bar, 0x3);
         }
         if (lane == 0) {
             int zero = 0;
