@@ -17,8 +17,16 @@
 // accumulator, and four epilogue warps read it back.  The rotation pairs row
 // r with row r ^ D/2 of the same head, which lives in another warp's TMEM
 // lanes, so the epilogue stages each 32-node slice of the tile in shared
-// memory, then every thread rotates its row against its partner and writes
-// bf16 to q or to the cache.
+// memory; then each warp takes 8 of the slice's nodes and each lane 4
+// consecutive rows of one of them, rotates them against their partners and
+// writes 8 bytes of bf16 to q or to the cache (a warp covers a node's 128
+// rows with 256 contiguous bytes).
+// When (tile, node group) CTAs alone would leave SMs idle (one 64-node tree:
+// 48 tiles for Qwen3-8B), a cluster of up to four CTAs splits K: each reduces
+// its share of d into its own TMEM, hands each 32-node slice of its partial
+// to the first CTA through distributed shared memory (bounded mbarrier
+// handshakes: ready on the first CTA, free on the others), and the first CTA
+// adds them and runs the epilogue.
 #include "jsv_internal.cuh"
 #include "sm100.cuh"
 
@@ -33,11 +41,13 @@ constexpr int kQMaxStages = 8;
 constexpr int kQTileM = 128;
 constexpr int kQKChunk = 64;
 constexpr uint32_t kQStageA = kQTileM * 128;
-constexpr int kQSmemBudget = 180 * 1024;
+constexpr int kQSmemBudget = 164 * 1024;
+constexpr int kQMaxWalk = 512 + 256;             // parents a group's depth walks can visit
 
 struct QkvParams {
     BatchArgs a;
     int d, rows_total, kchunks, group_nodes, box_rows, stages;
+    int ksplit;        // CTAs of a cluster splitting K (1: no cluster)
     uint32_t stage_bytes;
     const float *cos, *sin;
     int max_pos;
@@ -59,13 +69,20 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ volatile int ep_fail;
-    __shared__ float tile[32][kQTileM];          // one 32-node slice, column-major by node
+    __shared__ __align__(8) uint64_t slice_ready, slice_free;
+    __shared__ __align__(16) float tile[32][kQTileM];   // one 32-node slice, a row of 128 tile rows per node
+    __shared__ float xch[32][kQTileM];           // a K-split partial handed to the first CTA
     __shared__ int s_pos[256], s_row[256];
+    __shared__ int s_par[kQMaxWalk];
 
     const BatchArgs &a = p.a;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row0 = blockIdx.x * kQTileM;
+    // K split: CTA ks of the cluster reduces K-chunks [kc0, kc1); the first
+    // CTA adds the others' partials and runs the epilogue
+    const int ks = p.ksplit > 1 ? (int)cluster_ctarank() : 0;
+    const int kc0 = p.kchunks * ks / p.ksplit, kc1 = p.kchunks * (ks + 1) / p.ksplit;
+    const int row0 = (blockIdx.x / p.ksplit) * kQTileM;
     const int node0 = blockIdx.y * p.group_nodes;
     const int in_group = min(p.group_nodes, a.total_nodes - node0);
 
@@ -76,6 +93,8 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
         mbar_init(&accf_bar, 1);
         mbar_init(&drain_bar, 1);
+        mbar_init(&slice_ready, 4 * (p.ksplit > 1 ? p.ksplit - 1 : 1));  // the peers' epilogue warps
+        mbar_init(&slice_free, 4);                                       // the first CTA's epilogue warps
         abort_sh = 0;
         ep_fail = 0;
         fence_barrier_init();
@@ -85,7 +104,8 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         tmem_relinquish();
     }
     tc_fence_before();
-    __syncthreads();
+    if (p.ksplit > 1) cluster_sync();            // every CTA's barriers initialised
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
@@ -98,7 +118,7 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
-            for (int kc = 0; kc < p.kchunks; ++kc) {
+            for (int kc = kc0; kc < kc1; ++kc) {
                 if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh)) {
                     abort_sh = 1;
                     flag_error(a.dev_status, JSV_ERR_TIMEOUT);
@@ -130,7 +150,7 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int kc = 0; kc < p.kchunks; ++kc) {
+            for (int kc = kc0; kc < kc1; ++kc) {
                 if (!mbar_wait(&full_bar[stage], phase, &abort_sh)) {
                     abort_sh = 1;
                     flag_error(a.dev_status, JSV_ERR_TIMEOUT);
@@ -143,7 +163,7 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
 #pragma unroll
                 for (int kk = 0; kk < kQKChunk / 16; ++kk)
                     mma_bf16_ss(tmem, desc_kmajor_sw128(sa + kk * 32), desc_kmajor_sw128(sb + kk * 32), idn,
-                                (kc | kk) != 0);
+                                (kc > kc0 || kk > 0) ? 1u : 0u);
                 mma_commit(&empty_bar[stage]);
                 if (++stage == p.stages) { stage = 0; phase ^= 1; }
             }
@@ -159,20 +179,34 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         const int et = threadIdx.x - 64;             // 0..127
         const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
         // where each node of the group goes: request, position, physical cache row
-        for (int c = et; c < in_group; c += 128) {
-            const int t = node0 + c;
-            int lo = 0, hi = a.B - 1;                // request of node t (node_offsets is sorted)
+        auto request_of = [&](int t) {               // node_offsets is sorted
+            int lo = 0, hi = a.B - 1;
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
                 if (a.node_offsets[mid] <= t) lo = mid; else hi = mid - 1;
             }
+            return lo;
+        };
+        // The depth walks only visit nodes of the requests that overlap this
+        // group, [first such request's base, node0 + in_group): at most 512 +
+        // 256 entries, staged in shared memory with one coalesced load.
+        const int wbase = a.node_offsets[request_of(node0)];
+        const int wcount = node0 + in_group - wbase;
+        const bool staged = wbase >= 0 && wcount > 0 && wcount <= kQMaxWalk;
+        if (staged)
+            for (int i = et; i < wcount; i += 128) s_par[i] = __ldg(a.parent + wbase + i);
+        named_barrier(1, 128);
+        for (int c = et; c < in_group; c += 128) {
+            const int t = node0 + c;
+            const int lo = request_of(t);
             Request req;
             int pos = -1, row = -1;
             if (load_request(a, lo, req)) {
                 int j = t - req.base, dep = 0, steps = 0;
                 bool ok = true;
                 while (j > 0) {
-                    const int pj = a.parent[req.base + j];
+                    const int gi = req.base + j;
+                    const int pj = (staged && gi >= wbase && gi < wbase + wcount) ? s_par[gi - wbase] : a.parent[gi];
                     if (pj < 0 || pj >= j || ++steps > req.n) { ok = false; break; }
                     j = pj;
                     ++dep;
@@ -189,13 +223,7 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
         named_barrier(1, 128);
 
-        const int grow = row0 + r;                   // global W row of this thread
-        const int qrows = a.Hq * a.D, krows = a.Hkv * a.D;
-        const int kind = grow < qrows ? 0 : (grow < qrows + krows ? 1 : 2);   // Q, K, V
-        const int hrow = kind == 0 ? grow : (kind == 1 ? grow - qrows : grow - qrows - krows);
-        const int head = hrow / a.D, o = hrow % a.D, half = a.D / 2;
-        const int partner = r ^ half;
-        const bool rvalid = grow < p.rows_total;
+        const int qrows = a.Hq * a.D, krows = a.Hkv * a.D, half = a.D / 2;
 
         if (!mbar_wait(&accf_bar, 0, &abort_sh)) {
             abort_sh = 1;
@@ -205,30 +233,91 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         named_barrier(1, 128);
         if (!ep_fail) {
             tc_fence_after();
-            for (int c0 = 0; c0 < in_group; c0 += 32) {
+            for (int c0 = 0, sl = 0; c0 < in_group; c0 += 32, ++sl) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)c0, v);
                 tmem_ld_wait();
+                if (ks > 0) {
+                    // hand this slice to the first CTA (once it has taken the previous one)
+                    bool okw = sl == 0 || mbar_wait_cluster(&slice_free, (uint32_t)((sl - 1) & 1), &abort_sh);
+                    if (__any_sync(0xffffffffu, !okw)) {
+                        if (lane == 0) flag_error(a.dev_status, JSV_ERR_TIMEOUT);
+                        break;
+                    }
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) xch[x][r] = __uint_as_float(v[x]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&slice_ready, 0));
+                    continue;
+                }
+                if (p.ksplit > 1) {
+                    // add the other CTAs' partials of this slice, then release them
+                    bool okw = mbar_wait_cluster(&slice_ready, (uint32_t)(sl & 1), &abort_sh);
+                    if (__any_sync(0xffffffffu, !okw)) {
+                        if (lane == 0) flag_error(a.dev_status, JSV_ERR_TIMEOUT);
+                        break;
+                    }
+                    for (int q = 1; q < p.ksplit; ++q) {
+                        // all 32 remote loads in flight before the first add
+                        const uint32_t base = cluster_addr(&xch[0][r], (uint32_t)q);
+                        float pq[32];
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) pq[x] = ld_shared_cluster_f32(base + (uint32_t)(x * kQTileM * 4));
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) + pq[x]);
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        for (int q = 1; q < p.ksplit; ++q) mbar_arrive_cluster(cluster_addr(&slice_free, (uint32_t)q));
+                }
 #pragma unroll
                 for (int x = 0; x < 32; ++x) tile[x][r] = __uint_as_float(v[x]);
                 named_barrier(1, 128);
-                if (rvalid) {
-                    for (int x = 0; x < 32 && c0 + x < in_group; ++x) {
-                        const int c = c0 + x;
+                // Each warp takes 8 of the slice's 32 nodes (x = sub + 4k) and each
+                // lane 4 consecutive rows of the tile, so a warp writes a node's
+                // 128 rows as 256 contiguous bytes with one 8-byte store a lane.
+                // The slice's cos/sin loads are all issued before any is used.
+                {
+                    const int q0 = lane * 4;                        // tile rows q0 .. q0 + 3
+                    const int g0 = row0 + q0;
+                    const int kq = g0 < qrows ? 0 : (g0 < qrows + krows ? 1 : 2);   // Q, K, V
+                    const int hq = kq == 0 ? g0 : (kq == 1 ? g0 - qrows : g0 - qrows - krows);
+                    const int headq = hq / a.D, oq = hq % a.D, iq = oq % half;
+                    const bool qvalid = g0 + 3 < p.rows_total;
+                    float4 cs[8], sn[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int c = c0 + sub + 4 * k;
+                        const int pos = c < in_group ? s_pos[c] : -1;
+                        cs[k] = make_float4(1.f, 1.f, 1.f, 1.f);
+                        sn[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (kq < 2 && qvalid && pos >= 0) {
+                            cs[k] = __ldg(reinterpret_cast<const float4 *>(p.cos + (size_t)pos * half + iq));
+                            sn[k] = __ldg(reinterpret_cast<const float4 *>(p.sin + (size_t)pos * half + iq));
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int x = sub + 4 * k, c = c0 + x;
+                        if (c >= in_group || !qvalid) continue;
                         const int pos = s_pos[c], prow = s_row[c];
                         if (pos < 0 || prow < 0) continue;
-                        float val = tile[x][r];
-                        if (kind < 2) {
-                            const int i = o % half;
-                            const float cs = p.cos[(size_t)pos * half + i], sn = p.sin[(size_t)pos * half + i];
-                            const float pv = tile[x][partner];
-                            val = o < half ? fmaf(val, cs, -pv * sn) : fmaf(val, cs, pv * sn);
+                        float4 v = *reinterpret_cast<const float4 *>(&tile[x][q0]);
+                        if (kq < 2) {
+                            const float4 pv = *reinterpret_cast<const float4 *>(&tile[x][q0 ^ half]);
+                            const float sg = oq < half ? -1.f : 1.f;     // rotate-half sign
+                            v.x = fmaf(v.x, cs[k].x, sg * pv.x * sn[k].x);
+                            v.y = fmaf(v.y, cs[k].y, sg * pv.y * sn[k].y);
+                            v.z = fmaf(v.z, cs[k].z, sg * pv.z * sn[k].z);
+                            v.w = fmaf(v.w, cs[k].w, sg * pv.w * sn[k].w);
                         }
+                        uint2 pk;
+                        pk.x = (uint32_t)to_bf16_bits(v.x) | ((uint32_t)to_bf16_bits(v.y) << 16);
+                        pk.y = (uint32_t)to_bf16_bits(v.z) | ((uint32_t)to_bf16_bits(v.w) << 16);
                         const int t = node0 + c;
-                        const uint16_t hb = to_bf16_bits(val);
-                        if (kind == 0) p.q[((size_t)t * a.Hq + head) * a.D + o] = hb;
-                        else if (kind == 1) p.k_cache[((size_t)prow * a.Hkv + head) * a.D + o] = hb;
-                        else p.v_cache[((size_t)prow * a.Hkv + head) * a.D + o] = hb;
+                        uint16_t *dst = kq == 0 ? p.q + ((size_t)t * a.Hq + headq) * a.D + oq
+                                        : (kq == 1 ? p.k_cache : p.v_cache) + ((size_t)prow * a.Hkv + headq) * a.D + oq;
+                        *reinterpret_cast<uint2 *>(dst) = pk;
                     }
                 }
                 named_barrier(1, 128);
@@ -236,8 +325,10 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
     }
 
+    __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    if (p.ksplit > 1) cluster_sync();            // no CTA leaves while its partial may still be read
+    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, 256);
@@ -265,6 +356,7 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
     p.q = q;
     p.k_cache = k_cache;
     p.v_cache = v_cache;
+    p.ksplit = 1;
 
     CUtensorMap tmW, tmX;
     if (!encode_tensor_map_2d(&tmW, w_qkv, (uint64_t)d, (uint64_t)p.rows_total, (uint64_t)d * 2, kQKChunk, kQTileM))
@@ -281,8 +373,37 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    dim3 grid((p.rows_total + kQTileM - 1) / kQTileM, (a.total_nodes + p.group_nodes - 1) / p.group_nodes);
-    cudaError_t e = launch_pdl(qkv_rope_kernel, grid, dim3(kQThreads), smem, st, tmW, tmX, p);
+    const int tiles = (p.rows_total + kQTileM - 1) / kQTileM;
+    const int groups = (a.total_nodes + p.group_nodes - 1) / p.group_nodes;
+    // Too few (tile, group) CTAs to stream the weight with every SM: split K
+    // over a cluster of up to four CTAs (each keeping at least four chunks),
+    // as many as the SMs and the resident clusters allow.
+    const int sms = device_sm_count();
+    int ks = 1;
+    while (ks < 4 && (long long)tiles * groups * (ks + 1) <= sms && p.kchunks / (ks + 1) >= 4) ++ks;
+    for (; ks > 1; --ks) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(tiles * ks, groups);
+        cfg.blockDim = dim3(kQThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = ks;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, qkv_rope_kernel, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        if ((long long)n >= (long long)tiles * groups) break;     // one resident wave
+    }
+    p.ksplit = ks;
+    dim3 grid(tiles * ks, groups);
+    cudaError_t e = ks > 1 ? launch_pdl_cluster(qkv_rope_kernel, grid, dim3(kQThreads), smem, st, ks, tmW, tmX, p)
+                           : launch_pdl(qkv_rope_kernel, grid, dim3(kQThreads), smem, st, tmW, tmX, p);
     count_launches(1);
     return e;
 }
