@@ -9,8 +9,9 @@
 //     score descending, depth ascending, rank path (lexicographic) ascending,
 // which is ancestor- and sibling-closed, emitted breadth-first.
 //
-// One warp per request, no sorting and no heap:
-//  1. tau, the budget-th best score, by binary search over the fp32 order:
+// One CTA of 32 warps per request, no sorting and no heap:
+//  1. tau, the budget-th best score, by a 32-way search over the fp32 order
+//     (each round every warp tests one threshold, ~7 rounds instead of 32):
 //     count(x) = #nodes with score >= x comes from a level-by-level expansion
 //     that stops as soon as it reaches the budget (children of a node are
 //     scanned in rank order and stop at the first one below x, since the
@@ -59,19 +60,23 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
     return v;
 }
 
+constexpr int kTreeWarps = 32;                 // warps a request: one threshold each per round
+constexpr int kTreeLevel = kTreeMaxBudget + kTreeMaxWidth;
+
 struct TreeSmem {
     float lp[kTreeMaxDepth][kTreeMaxWidth];
-    float lvl[2][kTreeMaxBudget + kTreeMaxWidth];
     float nscore[kTreeMaxBudget];
     int32_t nparent[kTreeMaxBudget];
     uint8_t nrank[kTreeMaxBudget];
     uint8_t ndepth[kTreeMaxBudget];
+    int res[kTreeWarps];
+    uint32_t lo, hi;
+    int bad, take_all, nodes;
 };
 
 // Number of nodes with score >= x, capped at `cap` (exits as soon as it is
-// reached).  Warp-cooperative; the result is uniform.
-__device__ int count_ge(TreeSmem &sm, int D, int k, float x, int cap, int lane) {
-    float *cur = sm.lvl[0], *nxt = sm.lvl[1];
+// reached).  One warp, with its own two level buffers; the result is uniform.
+__device__ int count_ge(const TreeSmem &sm, float *cur, float *nxt, int D, int k, float x, int cap, int lane) {
     if (lane == 0) cur[0] = 0.f;
     __syncwarp();
     int ncur = 1, total = 1;
@@ -104,13 +109,14 @@ __device__ int count_ge(TreeSmem &sm, int D, int k, float x, int cap, int lane) 
     return total;
 }
 
-__global__ void __launch_bounds__(32)
+__global__ void __launch_bounds__(32 * kTreeWarps)
 accum_logp_tree_kernel(TreeArgs a) {
     pdl_allow_dependents();
     pdl_wait_predecessor();
     __shared__ TreeSmem sm;
-    const int b = blockIdx.x, lane = threadIdx.x;
-    int D = a.D;
+    extern __shared__ float lvl_all[];             // [kTreeWarps][2][kTreeLevel]
+    const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float *lvl0 = lvl_all + (size_t)warp * 2 * kTreeLevel, *lvl1 = lvl0 + kTreeLevel;
     const int k = a.k, budget = a.budget;
     int32_t *o_par = a.parent + (size_t)b * budget;
     int32_t *o_tok = a.tokens + (size_t)b * budget;
@@ -118,99 +124,131 @@ accum_logp_tree_kernel(TreeArgs a) {
     float *o_sc = a.score ? a.score + (size_t)b * budget : nullptr;
 
     // stage and validate the log-probs: finite or -inf, <= 0, non-increasing per depth
-    bool bad = false;
-    for (int e = lane; e < D * k; e += 32) {
-        const float v = a.logp[((size_t)b * D) * k + e];
-        const int r = e % k;
-        bad |= !(v <= 0.f) && !(v == -INFINITY);
-        sm.lp[e / k][r] = v;
+    if (threadIdx.x == 0) sm.bad = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.D * k; e += blockDim.x) {
+        const float v = a.logp[((size_t)b * a.D) * k + e];
+        if (!(v <= 0.f) && !(v == -INFINITY)) sm.bad = 1;
+        sm.lp[e / k][e % k] = v;
     }
-    __syncwarp();
-    for (int e = lane; e < D * k; e += 32) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < a.D * k; e += blockDim.x) {
         const int m = e / k, r = e % k;
-        if (r > 0 && !(sm.lp[m][r] <= sm.lp[m][r - 1])) bad = true;
+        if (r > 0 && !(sm.lp[m][r] <= sm.lp[m][r - 1])) sm.bad = 1;
     }
-    if (__any_sync(0xffffffffu, bad)) {
-        if (lane == 0) flag_error(a.status, JSV_ERR_DEVICE_INPUT);
+    __syncthreads();
+    int D = a.D;
+    if (sm.bad) {
+        if (threadIdx.x == 0) flag_error(a.status, JSV_ERR_DEVICE_INPUT);
         D = 0;    // emit the root alone
     }
 
-    // 1. tau: the largest x with count(x) >= budget, by bisection over the fp32 order
-    int take_all = 0;
-    uint32_t lo = f2ord(-INFINITY), hi = f2ord(0.f) + 1u;
-    if (budget <= 1 || D == 0) {
-        take_all = 0;
-        lo = f2ord(0.f);
-    } else if (count_ge(sm, D, k, -INFINITY, budget, lane) < budget) {
-        take_all = 1;                     // the whole candidate tree fits the budget
-    } else {
-        while (hi - lo > 1u) {
-            const uint32_t mid = lo + (hi - lo) / 2u;
-            if (count_ge(sm, D, k, ord2f(mid), budget, lane) >= budget) lo = mid;
-            else hi = mid;
+    // 1. tau: the largest x with count(x) >= budget.  Invariant count(lo) >=
+    //    budget > count(hi) over the fp32 order; each round warp w tests
+    //    lo + (hi - lo) * w / 32 and the interval shrinks to the last passing
+    //    point and the next (count is non-increasing in x).
+    if (threadIdx.x == 0) {
+        sm.lo = f2ord(-INFINITY);
+        sm.hi = f2ord(0.f) + 1u;
+        sm.take_all = 0;
+    }
+    __syncthreads();
+    const bool search = budget > 1 && D > 0;
+    if (search && warp == 0) {
+        const int all = count_ge(sm, lvl0, lvl1, D, k, -INFINITY, budget, lane);
+        if (lane == 0) sm.take_all = all < budget;   // the whole candidate tree fits the budget
+    }
+    __syncthreads();
+    if (search && !sm.take_all) {
+        while (sm.hi - sm.lo > 1u) {
+            const uint32_t lo = sm.lo, hi = sm.hi;
+            const uint32_t t = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)warp) >> 5);
+            const int ok = warp == 0 ? 1 : (count_ge(sm, lvl0, lvl1, D, k, ord2f(t), budget, lane) >= budget);
+            if (lane == 0) sm.res[warp] = ok;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                int w = kTreeWarps - 1;
+                while (w > 0 && !sm.res[w]) --w;
+                sm.lo = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)w) >> 5);
+                if (w + 1 < kTreeWarps)
+                    sm.hi = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)(w + 1)) >> 5);
+            }
+            __syncthreads();
         }
     }
+    if (!search) {
+        if (threadIdx.x == 0) sm.lo = f2ord(0.f);
+        __syncthreads();
+    }
+    const int take_all = search && sm.take_all;
+    const uint32_t lo = sm.lo;
     const float tau = take_all ? -INFINITY : ord2f(lo);
-    // nodes strictly above tau (uncapped count is < budget by the bisection)
-    int ties_left;
-    if (take_all) {
-        ties_left = budget;
-    } else if (budget <= 1 || D == 0) {
-        ties_left = 0;
-    } else {
-        const int n_gt = lo == f2ord(0.f) ? count_ge(sm, D, k, __uint_as_float(0x00000001u), budget, lane)
-                                          : count_ge(sm, D, k, ord2f(lo + 1u), budget, lane);
-        ties_left = budget - n_gt;
-    }
 
-    // 2. materialise level by level in breadth-first order
-    if (lane == 0) {
-        sm.nscore[0] = 0.f;
-        sm.nparent[0] = -1;
-        sm.nrank[0] = 0;
-        sm.ndepth[0] = 0;
-    }
-    __syncwarp();
-    int n = 1, lvl_begin = 0, lvl_end = 1;
-    for (int m = 0; m < D && lvl_begin < lvl_end && n < budget; ++m) {
-        for (int c0 = lvl_begin; c0 < lvl_end; c0 += 32) {
-            const int i = c0 + lane;
-            float s = 0.f;
-            int cgt = 0, ceq = 0;
-            if (i < lvl_end) {
-                s = sm.nscore[i];
-                for (int r = 0; r < k; ++r) {
-                    const float cs = __fadd_rn(s, sm.lp[m][r]);
-                    if (cs > tau) ++cgt;
-                    else if (cs == tau) ++ceq;
-                    else break;
-                }
-            }
-            // ties are taken in breadth-first order while the tie budget lasts
-            const int eq_incl = warp_incl_scan(ceq, lane);
-            const int eq_excl = eq_incl - ceq;
-            const int take_eq = max(0, min(ceq, ties_left - eq_excl));
-            const int c = cgt + take_eq;
-            const int incl = warp_incl_scan(c, lane);
-            const int tot = __shfl_sync(0xffffffffu, incl, 31);
-            const int used_eq = __shfl_sync(0xffffffffu, max(0, min(eq_incl, ties_left)), 31);
-            const int off = n + incl - c;
-            for (int r = 0; r < c && off + r < budget; ++r) {
-                sm.nscore[off + r] = __fadd_rn(s, sm.lp[m][r]);
-                sm.nparent[off + r] = i;
-                sm.nrank[off + r] = (uint8_t)r;
-                sm.ndepth[off + r] = (uint8_t)(m + 1);
-            }
-            n = min(budget, n + tot);
-            ties_left -= used_eq;
+    // 2. (warp 0) nodes strictly above tau, then materialise level by level
+    //    in breadth-first order
+    int n = 1;
+    if (warp == 0) {
+        int ties_left;
+        if (take_all) {
+            ties_left = budget;
+        } else if (!search) {
+            ties_left = 0;
+        } else {
+            const int n_gt = lo == f2ord(0.f) ? count_ge(sm, lvl0, lvl1, D, k, __uint_as_float(0x00000001u), budget, lane)
+                                              : count_ge(sm, lvl0, lvl1, D, k, ord2f(lo + 1u), budget, lane);
+            ties_left = budget - n_gt;
+        }
+        if (lane == 0) {
+            sm.nscore[0] = 0.f;
+            sm.nparent[0] = -1;
+            sm.nrank[0] = 0;
+            sm.ndepth[0] = 0;
         }
         __syncwarp();
-        lvl_begin = lvl_end;
-        lvl_end = n;
+        int lvl_begin = 0, lvl_end = 1;
+        for (int m = 0; m < D && lvl_begin < lvl_end && n < budget; ++m) {
+            for (int c0 = lvl_begin; c0 < lvl_end; c0 += 32) {
+                const int i = c0 + lane;
+                float s = 0.f;
+                int cgt = 0, ceq = 0;
+                if (i < lvl_end) {
+                    s = sm.nscore[i];
+                    for (int r = 0; r < k; ++r) {
+                        const float cs = __fadd_rn(s, sm.lp[m][r]);
+                        if (cs > tau) ++cgt;
+                        else if (cs == tau) ++ceq;
+                        else break;
+                    }
+                }
+                // ties are taken in breadth-first order while the tie budget lasts
+                const int eq_incl = warp_incl_scan(ceq, lane);
+                const int eq_excl = eq_incl - ceq;
+                const int take_eq = max(0, min(ceq, ties_left - eq_excl));
+                const int c = cgt + take_eq;
+                const int incl = warp_incl_scan(c, lane);
+                const int tot = __shfl_sync(0xffffffffu, incl, 31);
+                const int used_eq = __shfl_sync(0xffffffffu, max(0, min(eq_incl, ties_left)), 31);
+                const int off = n + incl - c;
+                for (int r = 0; r < c && off + r < budget; ++r) {
+                    sm.nscore[off + r] = __fadd_rn(s, sm.lp[m][r]);
+                    sm.nparent[off + r] = i;
+                    sm.nrank[off + r] = (uint8_t)r;
+                    sm.ndepth[off + r] = (uint8_t)(m + 1);
+                }
+                n = min(budget, n + tot);
+                ties_left -= used_eq;
+            }
+            __syncwarp();
+            lvl_begin = lvl_end;
+            lvl_end = n;
+        }
+        if (lane == 0) sm.nodes = n;              // node count for the other warps
     }
+    __syncthreads();
+    n = sm.nodes;
 
     // outputs; unused slots get parent -1, token -1, depth -1
-    for (int i = lane; i < budget; i += 32) {
+    for (int i = threadIdx.x; i < budget; i += blockDim.x) {
         if (i < n) {
             const int d = sm.ndepth[i];
             o_par[i] = sm.nparent[i];
@@ -225,14 +263,24 @@ accum_logp_tree_kernel(TreeArgs a) {
             if (o_sc) o_sc[i] = -INFINITY;
         }
     }
-    if (lane == 0) a.num_nodes[b] = n;
+    if (threadIdx.x == 0) a.num_nodes[b] = n;
 }
 
 cudaError_t launch_accum_logp_tree(const float *logp, const int32_t *topk_tokens, const int32_t *root_token, int B,
                                    int D, int k, int budget, int32_t *parent, int32_t *tokens, int32_t *depth,
                                    float *score, int32_t *num_nodes, int32_t *status, cudaStream_t st) {
     TreeArgs a{logp, topk_tokens, root_token, B, D, k, budget, parent, tokens, depth, score, num_nodes, status};
-    cudaError_t e = launch_pdl(accum_logp_tree_kernel, dim3(B), dim3(32), 0, st, a);
+    const size_t smem = (size_t)kTreeWarps * 2 * kTreeLevel * sizeof(float);
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(accum_logp_tree_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    cudaError_t e = launch_pdl(accum_logp_tree_kernel, dim3(B), dim3(32 * kTreeWarps), smem, st, a);
     count_launches(1);
     return e;
 }
