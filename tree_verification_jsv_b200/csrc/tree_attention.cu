@@ -10,9 +10,10 @@
 // row r <-> node r / G, head g*G + r % G, so every K/V tile loaded serves
 // 256 query rows (GQA packing).  The 256 rows form two 128-row groups that
 // take turns on the tensor core.  The prefix is cut into 128-key tiles that
-// start on page boundaries; split s takes a contiguous run of them, and the
-// last split also takes the tree tiles, which cover slots [P & ~15, P + N)
-// and apply the ancestor mask.  Each split writes an unnormalised fp32
+// start on page boundaries, followed by the tree tiles, which cover slots
+// [P & ~15, P + N) and apply the ancestor mask; split s takes a balanced
+// contiguous run of these tiles (a split that holds tree tiles builds the
+// ancestor bitsets).  Each split writes an unnormalised fp32
 // partial (O, row max, row sum); a small combine kernel merges the splits
 // with log-sum-exp rescaling and rounds to bf16.
 //
@@ -187,12 +188,15 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     const int ngroups = rows_here > kGroupRows ? 2 : 1;     // a group with no rows is skipped
 
     // tile schedule for this split
+    // Logical tiles: the prefix tiles, then the tree tiles; split s takes the
+    // balanced run [total * s / S, total * (s + 1) / S).
     const int prefix_tiles = (r.P + kKeyTile - 1) / kKeyTile;
-    const int t_begin = (int)((long long)prefix_tiles * split / prm.S);
-    const int t_end = (int)((long long)prefix_tiles * (split + 1) / prm.S);
     const int P0 = r.P & ~15;                    // tree tiles start on a page boundary
-    const int tree_tiles = (split == prm.S - 1) ? (r.P + r.n - P0 + kKeyTile - 1) / kKeyTile : 0;
-    const int ntiles = (t_end - t_begin) + tree_tiles;
+    const int total_tiles = prefix_tiles + (r.P + r.n - P0 + kKeyTile - 1) / kKeyTile;
+    const int t_begin = (int)((long long)total_tiles * split / prm.S);
+    const int t_end = (int)((long long)total_tiles * (split + 1) / prm.S);
+    const int ntiles = t_end - t_begin;
+    const int tree_tiles = max(0, t_end - max(t_begin, prefix_tiles));    // tree tiles of this split
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;
@@ -228,7 +232,8 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 
     // logical tile index -> first logical slot
     auto tile_slot0 = [&](int j) -> int {
-        return j < (t_end - t_begin) ? (t_begin + j) * kKeyTile : P0 + (j - (t_end - t_begin)) * kKeyTile;
+        const int lj = t_begin + j;
+        return lj < prefix_tiles ? lj * kKeyTile : P0 + (lj - prefix_tiles) * kKeyTile;
     };
 
     if (warp < kSoftmaxWarp0) {
@@ -521,7 +526,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             tc_fence_after();
             const int slot0 = tile_slot0(j);
-            const bool is_tree = j >= (t_end - t_begin);
+            const bool is_tree = t_begin + j >= prefix_tiles;
             const uint32_t sbase = tS + lane_addr;
             // The whole 128-column row of S in registers: one TMEM round trip.
             uint32_t sv[kKeyTile / 32][32];
@@ -769,24 +774,25 @@ tree_attention_combine_kernel(BatchArgs a, int S, const float *__restrict__ ws_o
 // Host side
 // ---------------------------------------------------------------------------
 static int attention_splits(const BatchArgs &a) {
-    // Split the prefix so the grid fills whole waves of SMs (1 CTA per SM),
-    // keeping at least two 128-key tiles per split.
+    // Choose S to minimise an estimate of the kernel time in tile periods
+    // (about 2.3 us each): waves(S) * (kFixed + ceil(total / S)) plus, per
+    // split, the write and read of its fp32 partial at about 6 TB/s, where
+    // total = prefix tiles + tree tiles of the largest request, a wave is one
+    // CTA per SM and kFixed covers set-up, the first loads and the partial
+    // write of a CTA.
     const int G = a.Hq / a.Hkv;
     const int mtiles = (a.max_nodes * G + kRowsPerCta - 1) / kRowsPerCta;
     const long long units = (long long)a.B * a.Hkv * mtiles;
-    const int prefix_tiles = (a.max_prefix + kKeyTile - 1) / kKeyTile;
-    int cap = prefix_tiles / 2;
-    if (cap < 1) cap = 1;
-    if (cap > 32) cap = 32;
+    const int total = (a.max_prefix + kKeyTile - 1) / kKeyTile + (a.max_nodes + 15 + kKeyTile - 1) / kKeyTile;
     const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+    const double kFixed = 3.0, kTileUs = 2.3;
+    const double comb = (double)a.total_nodes * a.Hq * (a.D + 2) * 4.0 * 2.0 / 6.0e6 / kTileUs;   // per split
     int best = 1;
-    double best_eff = -1.0;
-    for (int s = 1; s <= cap; ++s) {
-        const long long ctas = units * s;
-        const long long waves = (ctas + sms - 1) / sms;
-        const double eff = (double)ctas / (double)(waves * sms);
-        if (eff >= 0.9 && ctas >= sms) return s;
-        if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+    double best_cost = 1e300;
+    for (int s = 1; s <= 32 && s <= total; ++s) {
+        const long long waves = (units * s + sms - 1) / sms;
+        const double cost = (double)waves * (kFixed + (double)((total + s - 1) / s)) + (s > 1 ? s * comb : 0.0);
+        if (cost < best_cost - 1e-9) { best_cost = cost; best = s; }
     }
     return best;
 }
