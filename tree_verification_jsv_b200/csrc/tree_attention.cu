@@ -29,7 +29,8 @@
 //   warps 4..7  softmax of row group 0, warps 8..11 of row group 1: one query
 //               row per thread, the whole 128-column row of S read from TMEM
 //               into registers at once; masked online softmax in the log2
-//               domain; P_j (bf16) is written over its own S buffer in TMEM;
+//               domain (packed f32x2 arithmetic, three-input max); P_j (bf16)
+//               is written over its own S buffer in TMEM;
 //               O is rescaled in TMEM only when the running max grows by
 //               more than 8 (2^8), which keeps exp2 arguments bounded
 // While one group computes its softmax the tensor core runs the other
@@ -93,44 +94,12 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rm.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
 }
 
-// 2^x for a pair on the FMA pipe, to take part of the exponentials off the
-// MUFU unit: x = j + f with j = floor(x) (from adding 1.5 * 2^23 rounded
-// toward -inf), 2^f on [0, 1) from a cubic with p(0) = 1 whose coefficients
-// are a minimax fit of the relative error (8.6e-5, well below the bf16
-// rounding of P), and j added into the exponent field.  Inputs below -127
-// are clamped there, where the result is exactly +0; inputs are at most 8.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-    float x0, x1;
-    f2_unpack(x, x0, x1);
-    x = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
-    const uint64_t magic = f2_pack(12582912.f, 12582912.f);
-    const uint64_t t = f2_add_rm(x, magic);
-    const uint64_t f = f2_sub(x, f2_sub(t, magic));
-    uint64_t p = f2_fma(f2_pack(0.07706724f, 0.07706724f), f, f2_pack(0.22764498f, 0.22764498f));
-    p = f2_fma(p, f, f2_pack(0.69511663f, 0.69511663f));
-    p = f2_fma(p, f, f2_pack(1.f, 1.f));
-    float p0, p1, t0, t1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(t, t0, t1);
-    return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                   __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
-}
 
 struct AttnParams {
     BatchArgs a;
@@ -597,7 +566,9 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 
             // probabilities (masked columns hold -inf and give 0), their sum, and
             // the bf16 P row stored into the first 64 columns of this S buffer;
-            // pairs in packed fp32, one pair in four through the polynomial 2^x
+            // scale, offset and row sum on packed fp32 pairs.  (Moving part of
+            // the exponentials to a polynomial on the FMA pipe was measured
+            // slower: this loop is bound by instruction issue, not by MUFU.)
             const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
             const uint64_t sl2x2 = f2_pack(sl2, sl2), negmx2 = f2_pack(neg_m, neg_m);
             uint64_t ps2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
@@ -606,14 +577,9 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             for (int i = 0; i < kKeyTile / 2; ++i) {
                 const int c = (2 * i) / 32, x = (2 * i) % 32;
                 const uint64_t xa = f2_fma(f2_pack(__uint_as_float(sv[c][x]), __uint_as_float(sv[c][x + 1])), sl2x2, negmx2);
-                uint64_t ea;
-                if ((i & 3) == 3) {
-                    ea = exp2_poly_x2(xa);
-                } else {
-                    float u0, u1;
-                    f2_unpack(xa, u0, u1);
-                    ea = f2_pack(fast_exp2(u0), fast_exp2(u1));
-                }
+                float u0, u1;
+                f2_unpack(xa, u0, u1);
+                const uint64_t ea = f2_pack(fast_exp2(u0), fast_exp2(u1));
                 ps2[i & 1] = f2_add(ps2[i & 1], ea);
                 float a0, a1;
                 f2_unpack(ea, a0, a1);
