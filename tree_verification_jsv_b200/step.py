@@ -7,6 +7,9 @@ tree attention, LM head + argmax, accept walk, KV compaction.
 
 ``run_host`` is the end-to-end form: it copies the step's per-step inputs
 from pinned host memory, runs the step, and copies the accepted paths back.
+The per-step inputs (tree arrays, tokens, q, hidden) live in one device
+arena and the outputs (paths, lengths) in another, each mirrored by one
+pinned host buffer, so each direction is a single copy.
 
 ``capture`` records the four calls once into a CUDA graph (the engine the
 JetSpec README describes replays CUDA graphs for wall-clock latency); every
@@ -30,6 +33,28 @@ def _bf16(bits, device):
     return t.view(torch.bfloat16).to(device)
 
 
+class _Arena:
+    """Named arrays packed at 256-byte offsets in one device buffer, with a
+    pinned host mirror; ``dev[name]`` / ``host[name]`` are typed views."""
+
+    def __init__(self, fields, device):
+        # fields: name -> (shape, torch dtype)
+        self.layout, off = {}, 0
+        for name, (shape, dtype) in fields.items():
+            n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+            self.layout[name] = (off, n, shape, dtype)
+            off += (n + 255) // 256 * 256
+        self.nbytes = max(off, 256)
+        self.dev_buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+        self.host_buf = torch.zeros(self.nbytes, dtype=torch.uint8).pin_memory()
+        self.dev = {k: self._view(self.dev_buf, k) for k in self.layout}
+        self.host = {k: self._view(self.host_buf, k) for k in self.layout}
+
+    def _view(self, buf, name):
+        off, n, shape, dtype = self.layout[name]
+        return buf[off:off + n].view(dtype).view(shape)
+
+
 class VerifyStep:
     """Device state for one verify step of a workload (see ``synth.Workload``)."""
 
@@ -40,24 +65,37 @@ class VerifyStep:
         self.T, self.d, self.V = wl.T, wl.d, wl.V
         self.scale = wl.scale
         self.max_path = int(max_path or wl.max_nodes)
-        self.page_table = _i32(wl.page_table, dev)
-        self.prefix_len = _i32(wl.prefix_len, dev)
-        self.node_offsets = _i32(wl.node_offsets, dev)
-        self.parent = _i32(wl.parent, dev)
-        self.tokens = _i32(tokens, dev)
-        self.q = _bf16(wl.q, dev)
+        # per-step inputs in one arena (filled once here from the workload)
+        inputs = {"page_table": np.ascontiguousarray(wl.page_table, dtype=np.int32),
+                  "prefix_len": np.ascontiguousarray(wl.prefix_len, dtype=np.int32),
+                  "node_offsets": np.ascontiguousarray(wl.node_offsets, dtype=np.int32),
+                  "parent": np.ascontiguousarray(wl.parent, dtype=np.int32),
+                  "tokens": np.ascontiguousarray(tokens, dtype=np.int32),
+                  "q": np.ascontiguousarray(wl.q, dtype=np.uint16),
+                  "hidden": np.ascontiguousarray(wl.hidden, dtype=np.uint16)}
+        self._in = _Arena({k: (v.shape, torch.int32 if v.dtype == np.int32 else torch.bfloat16)
+                           for k, v in inputs.items()}, dev)
+        for k, v in inputs.items():
+            hv = self._in.host[k]
+            if v.dtype == np.int32:
+                hv.copy_(torch.from_numpy(v))
+            else:
+                hv.view(torch.int16).copy_(torch.from_numpy(v.view(np.int16)))
+        self._in.dev_buf.copy_(self._in.host_buf)
+        for k, t in self._in.dev.items():
+            setattr(self, k, t)
         self.k_cache = _bf16(wl.k_cache, dev)
         self.v_cache = _bf16(wl.v_cache, dev)
-        self.hidden = _bf16(wl.hidden, dev)
         self.w = _bf16(wl.w, dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.out = torch.empty((self.T, self.Hq, self.D), dtype=torch.bfloat16, device=dev)
         self.argmax = torch.empty(self.T, dtype=torch.int32, device=dev)
         self.max_logit = torch.empty(self.T, dtype=torch.float32, device=dev)
-        self.path = torch.empty((self.B, self.max_path), dtype=torch.int32, device=dev)
-        self.accept_len = torch.empty(self.B, dtype=torch.int32, device=dev)
-        self.bonus = torch.empty(self.B, dtype=torch.int32, device=dev)
-        self.new_len = torch.empty(self.B, dtype=torch.int32, device=dev)
+        # per-step outputs in one arena
+        self._out = _Arena({"path": ((self.B, self.max_path), torch.int32), "accept_len": ((self.B,), torch.int32),
+                            "bonus": ((self.B,), torch.int32), "new_len": ((self.B,), torch.int32)}, dev)
+        for k, t in self._out.dev.items():
+            setattr(self, k, t)
         self.batch = jsv.make_batch(
             B=self.B, Hq=self.Hq, Hkv=self.Hkv, D=self.D,
             max_pages_per_req=wl.page_table.shape[1], num_pages=wl.num_pages,
@@ -68,7 +106,6 @@ class VerifyStep:
         lws = jsv.jsv_lmhead_argmax_workspace_size(self.T, self.d, self.V)
         self.attn_ws = torch.empty(max(aws, 256), dtype=torch.uint8, device=dev)
         self.lm_ws = torch.empty(max(lws, 8), dtype=torch.uint8, device=dev)
-        self._pinned = None
         self._graph = None
 
     # -- the four calls -----------------------------------------------------
@@ -118,28 +155,21 @@ class VerifyStep:
 
     # -- end-to-end form ----------------------------------------------------
     def host_inputs(self):
-        """Pinned host copies of the per-step inputs (tree, tokens, q, hidden)."""
-        if self._pinned is None:
-            self._pinned = {k: getattr(self, k).cpu().pin_memory()
-                            for k in ("page_table", "prefix_len", "node_offsets", "parent",
-                                      "tokens", "q", "hidden")}
-            self._pinned_out = {k: torch.empty_like(getattr(self, k), device="cpu").pin_memory()
-                                for k in ("path", "accept_len", "bonus", "new_len")}
-        return self._pinned
+        """Pinned host views of the per-step inputs (tree arrays, tokens, q,
+        hidden); ``run_host`` copies all of them in one transfer."""
+        return self._in.host
 
     def h2d_bytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in self.host_inputs().values())
+        return self._in.nbytes
 
     def d2h_bytes(self) -> int:
-        self.host_inputs()
-        return sum(t.numel() * t.element_size() for t in self._pinned_out.values())
+        return self._out.nbytes
 
     def run_host(self, stream=None):
-        """Copy inputs host->device, run the step, copy the results back."""
-        src = self.host_inputs()
-        for k, t in src.items():
-            getattr(self, k).copy_(t, non_blocking=True)
+        """Copy the input arena host->device, run the step, copy the output
+        arena back (one copy each way); returns pinned host views of path,
+        accept_len, bonus and new_len."""
+        self._in.dev_buf.copy_(self._in.host_buf, non_blocking=True)
         self.run(stream)
-        for k, t in self._pinned_out.items():
-            t.copy_(getattr(self, k), non_blocking=True)
-        return self._pinned_out
+        self._out.host_buf.copy_(self._out.dev_buf, non_blocking=True)
+        return self._out.host
