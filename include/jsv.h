@@ -189,7 +189,17 @@ JSV_API size_t jsv_lmhead_argmax_workspace_size(int32_t T, int32_t d, int32_t V)
  *   argmax     device [T] int32
  *   max_logit  device [T] float (the fp32 maximum) or NULL
  *   workspace  device scratch of jsv_lmhead_argmax_workspace_size() bytes,
- *              8-B aligned; the call initialises it
+ *              8-B aligned, ZERO-FILLED before its first use (e.g. one
+ *              cudaMemsetAsync when it is allocated); every call leaves it
+ *              zero-filled again, so it is reused without clearing.  After a
+ *              call that failed on the device, zero it again.
+ * Ordering: the kernel reads `hidden` and `w` while the previous launch on
+ * the stream may still be running (it waits for that launch only before it
+ * touches the workspace and the outputs), so the tree-attention kernels of
+ * the same step run beside its main loop.  Kernels of other libraries are
+ * complete before it starts, as usual; only a buffer written by an earlier
+ * call of THIS library that may still be in flight (for instance
+ * jsv_tree_attention's `out`) must not be passed as `hidden` or `w`.
  * Supported: 1 <= T, d % 64 == 0, 64 <= d <= 16384, 1 <= V < 2^31.
  */
 JSV_API jsv_status jsv_lmhead_argmax(const uint16_t *hidden, const uint16_t *w,
@@ -246,7 +256,8 @@ JSV_API jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uin
  *     that device current) and caches it; make that first call before any
  *     stream capture.
  *   - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
- *     library routine.  Each call clears the keys it uses before its kernel.
+ *     library routine.  The array starts zeroed and every call leaves the
+ *     keys it used zeroed again.
  *   - Every call shares the one array, which keeps the last call's contents:
  *     calls whose kernels overlap on the GPU (different streams, or
  *     different host threads on one device) race and give wrong results.

@@ -103,7 +103,7 @@ def test_lmhead_argmax_shapes(T, d, V):
     assert ok.mean() > 0.8
     arg = torch.empty(T, dtype=torch.int32, device="cuda")
     ml = torch.empty(T, dtype=torch.float32, device="cuda")
-    ws = torch.empty(jsv.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(jsv.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
     jsv.jsv_lmhead_argmax(_dev_bf16(H), _dev_bf16(W), T, d, V, arg, ml, ws)
     torch.cuda.synchronize()
     g = arg.cpu().numpy()
@@ -112,13 +112,37 @@ def test_lmhead_argmax_shapes(T, d, V):
     assert np.allclose(ml.cpu().numpy()[ok], t1[ok], rtol=1e-4, atol=1e-5)
 
 
+def test_lmhead_workspace_reused_without_clearing():
+    """One workspace, zeroed once, serves back-to-back calls of different
+    shapes on one stream with no synchronisation in between: every call must
+    leave the keys and the completion counter zeroed for the next one."""
+    shapes = [(64, 256, 5000), (16, 256, 5000), (64, 256, 5000), (100, 128, 3001), (3, 128, 3001)]
+    ws = torch.zeros(jsv.jsv_lmhead_argmax_workspace_size(128, 256, 5000), dtype=torch.uint8, device="cuda")
+    runs = []
+    for i, (T, d, V) in enumerate(shapes):
+        rng = np.random.default_rng(500 + i)
+        H = bf16(rng.standard_normal((T, d)) / math.sqrt(d))
+        W = bf16(rng.standard_normal((V, d)) / math.sqrt(d))
+        arg = torch.empty(T, dtype=torch.int32, device="cuda")
+        dh, dw = _dev_bf16(H), _dev_bf16(W)
+        jsv.jsv_lmhead_argmax(dh, dw, T, d, V, arg, None, ws)
+        runs.append((H, W, arg, dh, dw))
+    torch.cuda.synchronize()
+    for H, W, arg, _, _ in runs:
+        a, t1, t2 = oracle.lmhead_top2(H, W)
+        ok, _ = oracle.certify_margin(H, W, a, t1, t2)
+        assert ok.mean() > 0.8
+        assert np.array_equal(arg.cpu().numpy()[ok], a[ok])
+    assert not ws.any().item()
+
+
 def test_lmhead_ties_take_smallest_index():
     d, V, T = 64, 700, 3
     W = np.zeros((V, d), dtype=np.float32)
     W[[17, 300, 650]] = 1.0 / 8          # exact ties for every node
     H = np.full((T, d), 1.0 / 8, dtype=np.float32)
     arg = torch.empty(T, dtype=torch.int32, device="cuda")
-    ws = torch.empty(jsv.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(jsv.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
     jsv.jsv_lmhead_argmax(_dev_bf16(bf16(H)), _dev_bf16(bf16(W)), T, d, V, arg, None, ws)
     torch.cuda.synchronize()
     assert arg.cpu().tolist() == [17, 17, 17]

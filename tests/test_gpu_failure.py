@@ -26,7 +26,7 @@ def test_bounded_wait_times_out_and_context_survives():
     H = (torch.randn(T, d, device="cuda", generator=g) / math.sqrt(d)).to(torch.bfloat16)
     W = (torch.randn(V, d, device="cuda", generator=g) / math.sqrt(d)).to(torch.bfloat16)
     arg = torch.empty(T, dtype=torch.int32, device="cuda")
-    ws = torch.empty(jsv.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(jsv.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
     jsv.jsv_lmhead_argmax(H, W, T, d, V, arg, None, ws)
     torch.cuda.synchronize()
     a = arg.cpu().numpy()

@@ -39,7 +39,7 @@ def _bf16_dev(rng, shape, scale):
 def _with_workspace(lib, H, W, T, d, V):
     arg = torch.full((T,), -7, dtype=torch.int32, device="cuda")
     ml = torch.zeros(T, dtype=torch.float32, device="cuda")
-    ws = torch.empty(lib.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(lib.jsv_lmhead_argmax_workspace_size(T, d, V), dtype=torch.uint8, device="cuda")
     st = lib.jsv_lmhead_argmax(H.data_ptr(), W.data_ptr(), T, d, V, arg.data_ptr(), ml.data_ptr(),
                                ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
     assert st == 0

@@ -10,22 +10,26 @@
 // the tree nodes are the N dimension (operand B = H, up to 256 nodes per
 // MMA), so a 64-node tree still fills M = 128.
 //
-// An item is one 128-row vocabulary tile x one group of up to 256 nodes.
-// Persistent kernel, one CTA per SM, 6 warps:
-//   warp 0      TMA producer: W tile (16-row boxes for a ragged tile) + H
-//               tile per 64-wide K chunk into a ring of shared-memory stages
+// An item is one vocabulary unit (up to 128 rows) x one group of up to 256
+// nodes.  One CTA per SM at a time, 6 warps:
+//   warp 0      TMA producer: the unit's W rows (one box) + the group's H
+//               rows per 64-wide K chunk into a ring of shared-memory stages;
+//               also asks cluster launch control for the next item
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator, per-column argmax
-//               across the 128 vocabulary rows (a transposing butterfly of
-//               64-bit keys), then one atomicMax per node
+//               across the unit's vocabulary rows (a transposing butterfly
+//               of 64-bit keys), kept per node in shared memory
 // Two accumulators alternate in TMEM, so the epilogue of one item overlaps
 // the main loop of the next.
-// Work split: with one node group (up to 256 nodes; W, the dominant byte
-// stream, is read exactly once) each CTA owns a contiguous, balanced
-// vocabulary range [V*c/G, V*(c+1)/G) whose ragged last tile loads only the
-// 16-row boxes it needs.  With several node groups the tensor pipe
-// dominates: each CTA takes a balanced contiguous range of the (tile, group)
-// items, group fastest, so consecutive items reuse the same W tile from L2.
+// Work split: the grid has one CTA per item; a running CTA that finishes an
+// item cancels a CTA that has not started and takes its item (cluster launch
+// control), so the items spread over whatever SMs are free -- the kernel
+// starts beside the attention kernels of the step and takes their SMs as
+// they finish.  Units are whole 16-row boxes, balanced so that with every SM
+// free each CTA gets the same number of rows.  With one node group (up to
+// 256 nodes) W, the dominant byte stream, is read exactly once; with several
+// the items are ordered group fastest, so CTAs working at the same time
+// share a W unit through L2.
 //
 // Node groups above 128 (tensor-bound) run on CTA pairs with 2-SM MMAs; see
 // the pair kernel below.
@@ -33,8 +37,11 @@
 // Cross-CTA reduction: a 64-bit key per node whose high word is the fp32
 // value mapped to an order-preserving unsigned integer and whose low word is
 // ~index; atomicMax keeps the largest value and, among equal values, the
-// smallest index.  The last CTA to finish (a counter in the workspace) writes
-// every node's argmax and maximum.
+// smallest index.  Each CTA merges its per-node maxima into the keys once,
+// after waiting for the previous launch on the stream (the main loop reads
+// only W and H, so it does not wait).  The CTA that completes the count of
+// finished work (a counter in the workspace) writes every node's argmax and
+// maximum and zeroes the keys and the counter for the next call.
 #include "jsv_internal.cuh"
 #include "sm100.cuh"
 
@@ -77,74 +84,80 @@ struct LmParams {
     int group_nodes;   // nodes per group (<= 256): the H box height
     int stages;
     uint32_t stage_bytes;
+    int units;         // single-CTA form: vocabulary units (see lm_unit)
+    int unit_b;        // 16-row boxes of a short unit
+    int unit_rem;      // units [0, unit_rem) take unit_b + 1 boxes
     unsigned long long *keys;
-    unsigned int *done;        // CTAs finished (zeroed with the keys before the launch)
+    unsigned int *done;        // work finished so far (zero between calls)
     int32_t *argmax;
     float *max_logit;
     int32_t *status;
 };
 
-// The k-th item of a CTA: vocabulary rows [row0, row0 + rows) and node group g.
-struct LmItem {
-    int row0, rows, g;
+// Single-CTA form: the vocabulary is cut into `units` runs of whole 16-row
+// boxes, unit_b or unit_b + 1 boxes each (at most 8 = one 128-row MMA tile),
+// with the unit count a multiple of the SM count where the vocabulary
+// allows; the last run may reach past V, where the tensor map fills zeros
+// and the epilogue ignores the rows.  An item is one unit x one node group
+// (group fastest); the grid has one CTA per item.
+struct LmUnit {
+    int row0, boxes;
 };
 
-struct LmWork {
-    int r0, r1;        // vocabulary range (one node group)
-    int it0;           // first global item (several node groups)
-    int items;
-
-    __device__ LmWork(const LmParams &p, int cta, int G) {
-        if (p.ngroups == 1) {
-            r0 = (int)((long long)p.V * cta / G);
-            r1 = (int)((long long)p.V * (cta + 1) / G);
-            it0 = 0;
-            items = (r1 - r0 + kTileM - 1) / kTileM;
-        } else {
-            const long long total = (long long)((p.V + kTileM - 1) / kTileM) * p.ngroups;
-            r0 = r1 = 0;
-            it0 = (int)(total * cta / G);
-            items = (int)(total * (cta + 1) / G) - it0;
-        }
+__device__ __forceinline__ LmUnit lm_unit(const LmParams &p, int u) {
+    LmUnit t;
+    const int big = p.unit_b + 1;
+    if (u < p.unit_rem) {
+        t.row0 = u * big * kBoxRowsW;
+        t.boxes = big;
+    } else {
+        t.row0 = (p.unit_rem * big + (u - p.unit_rem) * p.unit_b) * kBoxRowsW;
+        t.boxes = p.unit_b;
     }
-    __device__ LmItem item(const LmParams &p, int k) const {
-        LmItem t;
-        if (p.ngroups == 1) {
-            t.row0 = r0 + k * kTileM;
-            t.rows = min(kTileM, r1 - t.row0);
-            t.g = 0;
-        } else {
-            const int i = it0 + k, vt = i / p.ngroups;
-            t.row0 = vt * kTileM;
-            t.rows = min(kTileM, p.V - t.row0);
-            t.g = i - vt * p.ngroups;
-        }
-        return t;
-    }
-};
+    return t;
+}
 
 __device__ __forceinline__ void set_abort(volatile int *abort, int32_t *status) {
     *abort = 1;
     if (status) atomicCAS(status, 0, JSV_ERR_TIMEOUT);
 }
 
+// Answers of cluster launch control: the CTA's k-th item is blockIdx.x for
+// k = 0; the answer carrying item k + 1 lands in slot k % kClcSlots, in
+// phase (k / kClcSlots) & 1.  Every role reads every answer.
+constexpr int kClcSlots = 4;
+constexpr int kClcReaders = 2 + kEpiWarps;     // producer, MMA issuer, epilogue warps
+
+// Dynamic scheduling: a running CTA that finishes an item cancels a CTA of
+// the grid that has not started yet and takes its item instead, so CTAs
+// that start late (their SM was still held by an earlier kernel) end up
+// with fewer items and all finish together.  Completion is counted in items:
+// each CTA adds the items it took, and the CTA that brings the count to the
+// grid size reduces the keys.
 __global__ void __launch_bounds__(kLmThreads, 1)
-lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmW16,
+lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmWbig, const __grid_constant__ CUtensorMap tmWsmall,
                         const __grid_constant__ CUtensorMap tmH, const LmParams p) {
     pdl_allow_dependents();
-    pdl_wait_predecessor();
+    // With one node group, nothing before the final reduction touches memory
+    // that an earlier launch on the stream may still be using (W and hidden
+    // are only read; keys live in shared memory until then), so the wait for
+    // that launch moves to the reduction and the main loop overlaps it.
+    const bool late_wait = p.ngroups == 1;
+    if (!late_wait) pdl_wait_predecessor();
     extern __shared__ uint8_t dsmem[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
     __shared__ __align__(8) uint64_t accf_bar[2], acce_bar[2], drain_bar;
+    __shared__ __align__(8) uint64_t clc_full[kClcSlots], clc_empty[kClcSlots];
+    __shared__ __align__(16) uint4 clc_resp[kClcSlots];
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ volatile int ep_fail;
+    __shared__ int claimed_sh;
     __shared__ unsigned long long red[kEpiWarps][kMaxGroupNodes];
+    __shared__ unsigned long long best[kMaxGroupNodes];     // this CTA's best key per node (one group)
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const LmWork work(p, blockIdx.x, gridDim.x);
-    const int items = work.items;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -155,9 +168,14 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
             mbar_init(&accf_bar[a], 1);
             mbar_init(&acce_bar[a], kEpiWarps);
         }
+        for (int s = 0; s < kClcSlots; ++s) {
+            mbar_init(&clc_full[s], 1);
+            mbar_init(&clc_empty[s], kClcReaders);
+        }
         mbar_init(&drain_bar, 1);
         abort_sh = 0;
         ep_fail = 0;
+        claimed_sh = 1;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -165,8 +183,8 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmW);
-        prefetch_tensormap(&tmW16);
+        prefetch_tensormap(&tmWbig);
+        prefetch_tensormap(&tmWsmall);
         prefetch_tensormap(&tmH);
     }
     tc_fence_before();
@@ -184,12 +202,25 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
             int stage = 0;
             uint32_t phase = 0;
             long long issued = 0;
-            for (int it = 0; it < items && !abort_sh; ++it) {
-                const LmItem t = work.item(p, it);
-                const uint32_t tx = (uint32_t)p.group_nodes * 128 +
-                                    (t.rows == kTileM ? kStageA
-                                                      : (uint32_t)((t.rows + kBoxRowsW - 1) / kBoxRowsW) * (kBoxRowsW * 128));
-                const int node0 = t.g * p.group_nodes;
+            int item = blockIdx.x, claimed = 1;
+            int pend_slot = -1;                  // an answer still on its way
+            uint32_t pend_phase = 0;
+            for (int k = 0; !abort_sh; ++k) {
+                const int cs = k % kClcSlots;
+                const uint32_t cph = (uint32_t)(k / kClcSlots) & 1u;
+                // ask for the next item while this one streams in
+                if (!mbar_wait(&clc_empty[cs], cph ^ 1, &abort_sh)) {
+                    set_abort(&abort_sh, p.status);
+                    break;
+                }
+                mbar_arrive_expect_tx(&clc_full[cs], 16);
+                clc_try_cancel(&clc_resp[cs], &clc_full[cs]);
+                pend_slot = cs;
+                pend_phase = cph;
+                const LmUnit t = lm_unit(p, item / p.ngroups);
+                const int node0 = (item % p.ngroups) * p.group_nodes;
+                const CUtensorMap *mw = t.boxes == p.unit_b ? &tmWsmall : &tmWbig;
+                const uint32_t tx = (uint32_t)p.group_nodes * 128 + (uint32_t)t.boxes * (kBoxRowsW * 128);
                 bool ok = true;
                 for (int kc = 0; kc < p.kchunks; ++kc) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh)) {
@@ -198,24 +229,38 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
                         break;
                     }
                     uint8_t *sa = smem + (size_t)stage * p.stage_bytes;
-                    uint8_t *sb = sa + kStageA;
                     mbar_arrive_expect_tx(&full_bar[stage], tx);
-                    if (t.rows == kTileM) {
-                        tma_load_2d_hint(sa, &tmW, &full_bar[stage], kc * kKChunk, t.row0, pol_w);
-                    } else {
-                        for (int bx = 0; bx * kBoxRowsW < t.rows; ++bx)
-                            tma_load_2d_hint(sa + bx * (kBoxRowsW * 128), &tmW16, &full_bar[stage], kc * kKChunk,
-                                             t.row0 + bx * kBoxRowsW, pol_w);
-                    }
-                    tma_load_2d_hint(sb, &tmH, &full_bar[stage], kc * kKChunk, node0, pol_h);
+                    tma_load_2d_hint(sa, mw, &full_bar[stage], kc * kKChunk, t.row0, pol_w);
+                    tma_load_2d_hint(sa + kStageA, &tmH, &full_bar[stage], kc * kKChunk, node0, pol_h);
                     ++issued;
                     if (++stage == p.stages) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
+                if (!mbar_wait(&clc_full[cs], cph, &abort_sh)) {
+                    set_abort(&abort_sh, p.status);
+                    break;
+                }
+                pend_slot = -1;
+                int next = 0;
+                const bool got = clc_query(&clc_resp[cs], next);
+                fence_async_smem();
+                mbar_arrive(&clc_empty[cs]);
+                if (!got) break;
+                item = next;
+                ++claimed;
+            }
+            int zero = 0;
+            if (pend_slot >= 0) {
+                // an answer is still on its way: it must land before the CTA
+                // exits, and an item it carries counts as taken (unprocessed
+                // after an abort, but the completion count still closes)
+                if (mbar_wait(&clc_full[pend_slot], pend_phase, (volatile int *)&zero)) {
+                    int next = 0;
+                    if (clc_query(&clc_resp[pend_slot], next)) ++claimed;
+                }
             }
             if (abort_sh) {
                 // let every load still in flight land before the CTA exits
-                int zero = 0;
                 const long long back = issued < p.stages ? issued : p.stages;
                 int s = stage;
                 uint32_t ph = phase;
@@ -225,22 +270,24 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
                     mbar_wait(&full_bar[s], ph, (volatile int *)&zero);
                 }
             }
+            claimed_sh = claimed;
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            for (int it = 0; it < items && !abort_sh; ++it) {
-                const int acc = it & 1;
-                const uint32_t use = (uint32_t)(it >> 1);
+            int item = blockIdx.x;
+            for (int k = 0; !abort_sh; ++k) {
+                const int acc = k & 1;
+                const uint32_t use = (uint32_t)(k >> 1);
                 if (!mbar_wait(&acce_bar[acc], (use & 1) ^ 1, &abort_sh)) {
                     set_abort(&abort_sh, p.status);
                     break;
                 }
                 tc_fence_after();
-                const LmItem t = work.item(p, it);
-                const int in_group = min(p.group_nodes, p.T - t.g * p.group_nodes);
+                const int node0 = (item % p.ngroups) * p.group_nodes;
+                const int in_group = min(p.group_nodes, p.T - node0);
                 const uint32_t idn = idesc_bf16_f32(kTileM, (in_group + 15) & ~15, false, false);
                 const uint32_t d0 = tmem + (uint32_t)acc * 256u;
                 bool ok = true;
@@ -262,6 +309,17 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
                 }
                 if (!ok) break;
                 mma_commit(&accf_bar[acc]);
+                const int cs = k % kClcSlots;
+                if (!mbar_wait(&clc_full[cs], (uint32_t)(k / kClcSlots) & 1u, &abort_sh)) {
+                    set_abort(&abort_sh, p.status);
+                    break;
+                }
+                int next = 0;
+                const bool got = clc_query(&clc_resp[cs], next);
+                fence_async_smem();
+                mbar_arrive(&clc_empty[cs]);
+                if (!got) break;
+                item = next;
             }
             // every MMA issued above has finished before TMEM is released
             int zero = 0;
@@ -274,9 +332,11 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
         const int sub = warp & 3;                    // TMEM lanes this warp may access
         const uint32_t lane_addr = (uint32_t)(sub * 32) << 16;
         const int et = threadIdx.x - 64;             // 0..127
-        for (int it = 0; it < items; ++it) {
-            const int acc = it & 1;
-            const uint32_t use = (uint32_t)(it >> 1);
+        for (int c = et; c < kMaxGroupNodes; c += 32 * kEpiWarps) best[c] = 0ull;
+        int item = blockIdx.x;
+        for (int k = 0;; ++k) {
+            const int acc = k & 1;
+            const uint32_t use = (uint32_t)(k >> 1);
             if (!mbar_wait(&accf_bar[acc], use & 1, &abort_sh)) {
                 set_abort(&abort_sh, p.status);
                 ep_fail = 1;
@@ -284,10 +344,10 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
             named_barrier(1, 32 * kEpiWarps);
             if (ep_fail) break;
             tc_fence_after();
-            const LmItem t = work.item(p, it);
+            const LmUnit t = lm_unit(p, item / p.ngroups);
             const int v = t.row0 + sub * 32 + lane;
-            const bool vvalid = v < t.row0 + t.rows;
-            const int node0 = t.g * p.group_nodes;
+            const bool vvalid = v < min(t.row0 + t.boxes * kBoxRowsW, p.V);
+            const int node0 = (item % p.ngroups) * p.group_nodes;
             const int in_group = min(p.group_nodes, p.T - node0);
             const int ncols = (in_group + 31) & ~31;
             const uint32_t base = tmem + lane_addr + (uint32_t)acc * 256u;
@@ -317,12 +377,37 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
             if (lane == 0) mbar_arrive(&acce_bar[acc]);
             named_barrier(1, 32 * kEpiWarps);
             for (int c = et; c < in_group; c += 32 * kEpiWarps) {
-                unsigned long long k = red[0][c];
+                unsigned long long key = red[0][c];
 #pragma unroll
-                for (int w = 1; w < kEpiWarps; ++w) k = umax64(k, red[w][c]);
-                if (k) atomicMax(&p.keys[node0 + c], k);
+                for (int w = 1; w < kEpiWarps; ++w) key = umax64(key, red[w][c]);
+                if (late_wait)
+                    best[c] = umax64(best[c], key);
+                else if (key)
+                    atomicMax(&p.keys[node0 + c], key);
+            }
+            // the next item (every epilogue warp reads the same answer)
+            const int cs = k % kClcSlots;
+            int next = 0;
+            bool got = false;
+            if (mbar_wait(&clc_full[cs], (uint32_t)(k / kClcSlots) & 1u, &abort_sh)) {
+                got = clc_query(&clc_resp[cs], next);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&clc_empty[cs]);
+            } else {
+                set_abort(&abort_sh, p.status);
+                ep_fail = 1;
             }
             named_barrier(1, 32 * kEpiWarps);
+            if (ep_fail || !got) break;
+            item = next;
+        }
+        if (late_wait) {
+            // the previous launch on the stream has completed: the keys are
+            // free (and zero), so this CTA's maxima go out now
+            pdl_wait_predecessor();
+            for (int c = et; c < p.T; c += 32 * kEpiWarps)
+                if (best[c]) atomicMax(&p.keys[c], best[c]);
         }
     }
 
@@ -333,17 +418,23 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
-    // the last CTA to finish turns every node's key into its argmax
+    // The CTA that completes the item count turns every node's key into its
+    // argmax and leaves the workspace zeroed for the next call.
     __shared__ int is_last;
-    if (threadIdx.x == 0) is_last = atomicAdd(p.done, 1u) == (unsigned)(gridDim.x - 1);
+    if (threadIdx.x == 0) {
+        const unsigned total = (unsigned)p.units * (unsigned)p.ngroups;
+        is_last = atomicAdd(p.done, (unsigned)claimed_sh) + (unsigned)claimed_sh == total;
+    }
     __syncthreads();
     if (is_last) {
+        pdl_wait_predecessor();
         __threadfence();
         for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
-            const unsigned long long k = atomicAdd(&p.keys[t], 0ull);
-            p.argmax[t] = (int32_t)(~(uint32_t)(k & 0xffffffffull));
-            if (p.max_logit) p.max_logit[t] = key_value(k);
+            const unsigned long long key = atomicExch(&p.keys[t], 0ull);
+            p.argmax[t] = (int32_t)(~(uint32_t)(key & 0xffffffffull));
+            if (p.max_logit) p.max_logit[t] = key_value(key);
         }
+        if (threadIdx.x == 0) atomicExch(p.done, 0u);
     }
 }
 
@@ -636,17 +727,19 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
         tc_fence_after();
         tmem_dealloc_pair(tmem, 512);
     }
-    // the last CTA to finish turns every node's key into its argmax
+    // the last CTA to finish turns every node's key into its argmax and
+    // leaves the workspace zeroed for the next call
     __shared__ int is_last;
     if (threadIdx.x == 0) is_last = atomicAdd(p.done, 1u) == (unsigned)(gridDim.x - 1);
     __syncthreads();
     if (is_last) {
         __threadfence();
         for (int t = threadIdx.x; t < p.T; t += blockDim.x) {
-            const unsigned long long k = atomicAdd(&p.keys[t], 0ull);
+            const unsigned long long k = atomicExch(&p.keys[t], 0ull);
             p.argmax[t] = (int32_t)(~(uint32_t)(k & 0xffffffffull));
             if (p.max_logit) p.max_logit[t] = key_value(k);
         }
+        if (threadIdx.x == 0) atomicExch(p.done, 0u);
     }
 }
 
@@ -732,8 +825,9 @@ cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int 
     if (!encode_tensor_map_2d(&tmH, hidden, (uint64_t)d, (uint64_t)T, (uint64_t)d * 2, kKChunk, h_box))
         return cudaErrorInvalidValue;
 
-    cudaError_t e = cudaMemsetAsync(keys, 0, lmhead_workspace_bytes(T, d, V), st);
-    if (e != cudaSuccess) return e;
+    // The workspace arrives zeroed (first use) or as the previous call left
+    // it (zeroed by that call's last CTA), so no clearing launch is needed.
+    cudaError_t e = cudaSuccess;
     if (use_pair) {
         p.stage_bytes = pair_stage;
         p.stages = pair_stages;
@@ -747,10 +841,25 @@ cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int 
         p.stages = kSmemBudget / (int)p.stage_bytes;
         if (p.stages > kMaxStages) p.stages = kMaxStages;
         const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
-        const long long items = (long long)((V + kTileM - 1) / kTileM) * p.ngroups;
-        int grid = sms;
-        if (grid > items) grid = (int)items;
-        e = launch_pdl(lmhead_argmax_tc_kernel, dim3(grid), dim3(kLmThreads), smem, st, tmW, tmW16, tmH, p);
+        // vocabulary units of whole 16-row boxes, at most 8 per unit, as many
+        // units per SM as that needs
+        const long long boxes = ((long long)V + kBoxRowsW - 1) / kBoxRowsW;
+        const long long per_sm = (boxes + 8LL * sms - 1) / (8LL * sms);
+        long long units = per_sm * sms;
+        if (units > boxes) units = boxes;
+        if (units * p.ngroups > 0x7fffffffLL) return cudaErrorInvalidValue;
+        p.units = (int)units;
+        p.unit_b = (int)(boxes / units);
+        p.unit_rem = (int)(boxes - (long long)p.unit_b * units);
+        const int big_rows = (p.unit_b + 1 < kTileM / kBoxRowsW ? p.unit_b + 1 : kTileM / kBoxRowsW) * kBoxRowsW;
+        CUtensorMap tmWbig, tmWsmall;
+        if (!encode_tensor_map_2d(&tmWbig, w, (uint64_t)d, (uint64_t)V, (uint64_t)d * 2, kKChunk, big_rows))
+            return cudaErrorInvalidValue;
+        if (!encode_tensor_map_2d(&tmWsmall, w, (uint64_t)d, (uint64_t)V, (uint64_t)d * 2, kKChunk,
+                                  p.unit_b * kBoxRowsW))
+            return cudaErrorInvalidValue;
+        e = launch_pdl(lmhead_argmax_tc_kernel, dim3((unsigned)(units * p.ngroups)), dim3(kLmThreads), smem, st,
+                       tmWbig, tmWsmall, tmH, p);
     }
     count_launches(1);
     return e;

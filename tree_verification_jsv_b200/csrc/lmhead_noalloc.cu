@@ -59,7 +59,7 @@ jsv_status jsv_lmhead_argmax_noalloc(const uint16_t *hidden, const uint16_t *w, 
         return JSV_ERR_INVALID_ARG;
     void *scratch = nullptr;
     if (jsv::noalloc_scratch(&scratch) != cudaSuccess) return JSV_ERR_CUDA;
-    // the launcher clears the keys and counter it uses before the kernel runs
+    // the array is zero at load and every call leaves its keys and counter zeroed
     static_assert(sizeof(jsv::g_lmhead_noalloc_keys) >= (JSV_NOALLOC_MAX_NODES + 1) * sizeof(unsigned long long),
                   "scratch must hold the keys and the completion counter");
     cudaError_t e = jsv::launch_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, scratch,

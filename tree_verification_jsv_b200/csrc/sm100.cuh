@@ -431,6 +431,38 @@ __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------ cluster launch control
+// Ask the hardware to cancel one CTA of this grid that has not started yet.
+// The 16-byte answer is written to `resp` (16-B aligned shared memory) and
+// completes `bar` with 16 transaction bytes, so the caller arms `bar` with
+// an expected byte count of 16 first.  No request may follow an answer that
+// reported no cancellation.
+__device__ __forceinline__ void clc_try_cancel(void *resp, uint64_t *bar) {
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+            smem_addr(resp)),
+        "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Read an answer: true, and the x index of the cancelled CTA, when a CTA was
+// cancelled (its work now belongs to the caller).
+__device__ __forceinline__ bool clc_query(const void *resp, int &ctaid_x) {
+    uint32_t x, ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b128 r;\n\t"
+        "mov.u32 %0, 0;\n\t"
+        "ld.shared.b128 r, [%2];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "selp.u32 %1, 1, 0, p;\n\t"
+        "@p clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%0, _, _, _}, r;\n\t}"
+        : "=r"(x), "=r"(ok)
+        : "r"(smem_addr(resp))
+        : "memory");
+    ctaid_x = (int)x;
+    return ok != 0;
+}
+
 }  // namespace sm100
 
 // Host side: tensor-map encoding through the driver entry point (no -lcuda).

@@ -105,7 +105,7 @@ class VerifyStep:
         aws = jsv.jsv_tree_attention_workspace_size(self.batch)
         lws = jsv.jsv_lmhead_argmax_workspace_size(self.T, self.d, self.V)
         self.attn_ws = torch.empty(max(aws, 256), dtype=torch.uint8, device=dev)
-        self.lm_ws = torch.empty(max(lws, 8), dtype=torch.uint8, device=dev)
+        self.lm_ws = torch.zeros(max(lws, 8), dtype=torch.uint8, device=dev)   # zeroed once; each call leaves it zeroed
         self._graph = None
 
     # -- the four calls -----------------------------------------------------
