@@ -84,7 +84,10 @@ cudaError_t launch_accept_path(const BatchArgs &a, const int32_t *tokens, const 
                                int max_path, int32_t *path, int32_t *accept_len, int32_t *bonus,
                                cudaStream_t st) {
     dim3 grid((a.B + kWalkWarps - 1) / kWalkWarps);
-    cudaError_t e = launch_pdl(accept_path_kernel, grid, dim3(kWalkWarps * 32), 0, st, a, tokens, argmax, max_path,
+    static bool carve[64] = {};
+    cudaError_t e = prefer_max_shared(accept_path_kernel, carve);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(accept_path_kernel, grid, dim3(kWalkWarps * 32), 0, st, a, tokens, argmax, max_path,
                                path, accept_len, bonus);
     count_launches(1);
     return e;

@@ -26,6 +26,25 @@ inline BatchArgs to_args(const jsv_batch *b) {
     return a;
 }
 
+// Kernels of a step run side by side on one SM (programmatic dependent
+// launch lets the next kernel start early), but an SM's split between L1 and
+// shared memory stays fixed while any CTA is resident on it.  A small kernel
+// left to the driver's default split would take a large L1 and keep the
+// LM-head and attention CTAs, which need most of the shared memory, off every
+// SM it occupies until it exits.  So every kernel asks for the largest shared
+// carveout; `done` is the call site's once-per-device flag array.
+template <typename K>
+inline cudaError_t prefer_max_shared(K *kernel, bool (&done)[64]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess) done[dev] = true;
+    return e;
+}
+
 // Programmatic dependent launch: every kernel of the library is launched so
 // that the next kernel in the stream may be scheduled before it finishes.
 // A kernel lets its dependents be scheduled at entry (they can only start

@@ -93,7 +93,10 @@ cudaError_t launch_kv_compact(const BatchArgs &a, uint16_t *k_cache, uint16_t *v
                               int32_t *new_len, cudaStream_t st) {
     dim3 grid(a.B, 2, (a.Hkv + kHeadsPerCta - 1) / kHeadsPerCta);
     size_t smem = (size_t)kCompactChunk * kHeadsPerCta * (a.D / 8) * sizeof(uint4);
-    cudaError_t e = launch_pdl(kv_compact_kernel, grid, dim3(kCompactThreads), smem, st, a, k_cache, v_cache, path,
+    static bool carve[64] = {};
+    cudaError_t e = prefer_max_shared(kv_compact_kernel, carve);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(kv_compact_kernel, grid, dim3(kCompactThreads), smem, st, a, k_cache, v_cache, path,
                                max_path, accept_len, new_len);
     count_launches(1);
     return e;

@@ -799,6 +799,12 @@ cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int 
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(lmhead_argmax_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kSmemBudget + 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(lmhead_argmax_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(lmhead_argmax_pair_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }

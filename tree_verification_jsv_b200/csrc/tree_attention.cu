@@ -674,10 +674,13 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 // ---------------------------------------------------------------------------
 // Split combine: one warp per (node, head) row.
 // ---------------------------------------------------------------------------
-constexpr int kCombineWarps = 8;
+// Small CTAs with at most 32 registers a thread: the combine grid becomes
+// resident (and waits) while the attention kernel runs, and must leave room
+// beside itself for the LM-head CTAs that start on the same SMs.
+constexpr int kCombineWarps = 4;
 
 template <int D>
-__global__ void __launch_bounds__(kCombineWarps * 32)
+__global__ void __launch_bounds__(kCombineWarps * 32, 16)
 tree_attention_combine_kernel(BatchArgs a, int S, const float *__restrict__ ws_o,
                               const float *__restrict__ ws_ml, uint16_t *__restrict__ out) {
     pdl_allow_dependents();
@@ -802,6 +805,9 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         cudaError_t e = cudaFuncSetAttribute(tree_attention_tc_kernel<D>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(tree_attention_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
@@ -815,6 +821,9 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
         return le;
     }
     dim3 cgrid((a.max_nodes * G + kCombineWarps - 1) / kCombineWarps, 1, a.B * a.Hkv);
+    static bool carve[64] = {};
+    le = prefer_max_shared(tree_attention_combine_kernel<D>, carve);
+    if (le != cudaSuccess) return le;
     le = launch_pdl(tree_attention_combine_kernel<D>, cgrid, dim3(kCombineWarps * 32), 0, st, a, S,
                     (const float *)prm.ws_o, (const float *)prm.ws_ml, out);
     count_launches(2);

@@ -277,6 +277,9 @@ cudaError_t launch_accum_logp_tree(const float *logp, const int32_t *topk_tokens
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         cudaError_t e = cudaFuncSetAttribute(accum_logp_tree_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(accum_logp_tree_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
