@@ -87,6 +87,7 @@ struct LmParams {
     int units;         // single-CTA form: vocabulary units (see lm_unit)
     int unit_b;        // 16-row boxes of a short unit
     int unit_rem;      // units [0, unit_rem) take unit_b + 1 boxes
+    int tiles;         // single-CTA form: 128-row W tiles a unit may span (1 or 2)
     unsigned long long *keys;
     unsigned int *done;        // work finished so far (zero between calls)
     int32_t *argmax;
@@ -95,13 +96,25 @@ struct LmParams {
 };
 
 // Single-CTA form: the vocabulary is cut into `units` runs of whole 16-row
-// boxes, unit_b or unit_b + 1 boxes each (at most 8 = one 128-row MMA tile),
-// with the unit count a multiple of the SM count where the vocabulary
-// allows; the last run may reach past V, where the tensor map fills zeros
-// and the epilogue ignores the rows.  An item is one unit x one node group
-// (group fastest); the grid has one CTA per item.
+// boxes, unit_b or unit_b + 1 boxes each, at most 8 per 128-row MMA tile and
+// `tiles` tiles per unit, with the unit count a multiple of the SM count
+// where the vocabulary allows; the last run may reach past V, where the
+// tensor map fills zeros and the epilogue ignores the rows.  An item is one
+// unit x one node group (group fastest); the grid has one CTA per item.
+//
+// Two tiles per unit: every K-chunk stage holds both tiles' W rows and ONE
+// copy of the group's H rows, and each K-step issues one MMA per tile into
+// its own TMEM accumulator.  The cost of a unit is set mostly by its K-chunk
+// stages (each brings the group's H rows from L2 and takes a full barrier
+// round trip), not by its W rows, so a unit twice as tall halves that cost
+// per vocabulary row.
 struct LmUnit {
     int row0, boxes;
+};
+
+// W tensor maps with box heights of 1..8 16-row boxes (one per height).
+struct LmWMaps {
+    CUtensorMap m[kTileM / kBoxRowsW];
 };
 
 __device__ __forceinline__ LmUnit lm_unit(const LmParams &p, int u) {
@@ -135,8 +148,8 @@ constexpr int kClcReaders = 2 + kEpiWarps;     // producer, MMA issuer, epilogue
 // each CTA adds the items it took, and the CTA that brings the count to the
 // grid size reduces the keys.
 __global__ void __launch_bounds__(kLmThreads, 1)
-lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmWbig, const __grid_constant__ CUtensorMap tmWsmall,
-                        const __grid_constant__ CUtensorMap tmH, const LmParams p) {
+lmhead_argmax_tc_kernel(const __grid_constant__ LmWMaps tmW, const __grid_constant__ CUtensorMap tmH,
+                        const LmParams p) {
     pdl_allow_dependents();
     // With one node group, nothing before the final reduction touches memory
     // that an earlier launch on the stream may still be using (W and hidden
@@ -183,8 +196,7 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmWbig, const __grid
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmWbig);
-        prefetch_tensormap(&tmWsmall);
+        for (int i = 0; i < kTileM / kBoxRowsW; ++i) prefetch_tensormap(&tmW.m[i]);
         prefetch_tensormap(&tmH);
     }
     tc_fence_before();
@@ -219,7 +231,7 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmWbig, const __grid
                 pend_phase = cph;
                 const LmUnit t = lm_unit(p, item / p.ngroups);
                 const int node0 = (item % p.ngroups) * p.group_nodes;
-                const CUtensorMap *mw = t.boxes == p.unit_b ? &tmWsmall : &tmWbig;
+                const int boxes0 = min(t.boxes, kTileM / kBoxRowsW), boxes1 = t.boxes - boxes0;
                 const uint32_t tx = (uint32_t)p.group_nodes * 128 + (uint32_t)t.boxes * (kBoxRowsW * 128);
                 bool ok = true;
                 for (int kc = 0; kc < p.kchunks; ++kc) {
@@ -230,8 +242,11 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmWbig, const __grid
                     }
                     uint8_t *sa = smem + (size_t)stage * p.stage_bytes;
                     mbar_arrive_expect_tx(&full_bar[stage], tx);
-                    tma_load_2d_hint(sa, mw, &full_bar[stage], kc * kKChunk, t.row0, pol_w);
-                    tma_load_2d_hint(sa + kStageA, &tmH, &full_bar[stage], kc * kKChunk, node0, pol_h);
+                    tma_load_2d_hint(sa, &tmW.m[boxes0 - 1], &full_bar[stage], kc * kKChunk, t.row0, pol_w);
+                    if (boxes1 > 0)
+                        tma_load_2d_hint(sa + kStageA, &tmW.m[boxes1 - 1], &full_bar[stage], kc * kKChunk,
+                                         t.row0 + kTileM, pol_w);
+                    tma_load_2d_hint(sa + p.tiles * kStageA, &tmH, &full_bar[stage], kc * kKChunk, node0, pol_h);
                     ++issued;
                     if (++stage == p.stages) { stage = 0; phase ^= 1; }
                 }
@@ -290,6 +305,8 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmWbig, const __grid
                 const int in_group = min(p.group_nodes, p.T - node0);
                 const uint32_t idn = idesc_bf16_f32(kTileM, (in_group + 15) & ~15, false, false);
                 const uint32_t d0 = tmem + (uint32_t)acc * 256u;
+                // a unit's second tile (rows 128..) accumulates 128 columns on
+                const bool two = lm_unit(p, item / p.ngroups).boxes > kTileM / kBoxRowsW;
                 bool ok = true;
                 for (int kc = 0; kc < p.kchunks; ++kc) {
                     if (!mbar_wait(&full_bar[stage], phase, &abort_sh)) {
@@ -299,11 +316,15 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmWbig, const __grid
                     }
                     tc_fence_after();
                     const uint32_t sa = smem_addr(smem + (size_t)stage * p.stage_bytes);
-                    const uint32_t sb = sa + kStageA;
+                    const uint32_t sb = sa + (uint32_t)p.tiles * kStageA;
 #pragma unroll
-                    for (int kk = 0; kk < kKChunk / 16; ++kk)
-                        mma_bf16_ss(d0, desc_kmajor_sw128(sa + kk * 32), desc_kmajor_sw128(sb + kk * 32), idn,
-                                    (kc | kk) != 0);
+                    for (int kk = 0; kk < kKChunk / 16; ++kk) {
+                        const uint64_t db = desc_kmajor_sw128(sb + kk * 32);
+                        mma_bf16_ss(d0, desc_kmajor_sw128(sa + kk * 32), db, idn, (kc | kk) != 0);
+                        if (two)
+                            mma_bf16_ss(d0 + (uint32_t)kTileM, desc_kmajor_sw128(sa + kStageA + kk * 32), db, idn,
+                                        (kc | kk) != 0);
+                    }
                     mma_commit(&empty_bar[stage]);
                     if (++stage == p.stages) { stage = 0; phase ^= 1; }
                 }
@@ -345,32 +366,36 @@ lmhead_argmax_tc_kernel(const __grid_constant__ CUtensorMap tmWbig, const __grid
             if (ep_fail) break;
             tc_fence_after();
             const LmUnit t = lm_unit(p, item / p.ngroups);
-            const int v = t.row0 + sub * 32 + lane;
-            const bool vvalid = v < min(t.row0 + t.boxes * kBoxRowsW, p.V);
+            const int row_end = min(t.row0 + t.boxes * kBoxRowsW, p.V);
+            const int ntiles = t.boxes > kTileM / kBoxRowsW ? 2 : 1;
             const int node0 = (item % p.ngroups) * p.group_nodes;
             const int in_group = min(p.group_nodes, p.T - node0);
             const int ncols = (in_group + 31) & ~31;
-            const uint32_t base = tmem + lane_addr + (uint32_t)acc * 256u;
-            for (int c0 = 0; c0 < ncols; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(base + (uint32_t)c0, r);
-                tmem_ld_wait();
-                unsigned long long x[32];
+            for (int tile = 0; tile < ntiles; ++tile) {
+                const int v = t.row0 + tile * kTileM + sub * 32 + lane;
+                const bool vvalid = v < row_end;
+                const uint32_t base = tmem + lane_addr + (uint32_t)acc * 256u + (uint32_t)(tile * kTileM);
+                for (int c0 = 0; c0 < ncols; c0 += 32) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(base + (uint32_t)c0, r);
+                    tmem_ld_wait();
+                    unsigned long long x[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    x[j] = (vvalid && c0 + j < in_group) ? argmax_key(__uint_as_float(r[j]), v) : 0ull;
-                // transposing butterfly: afterwards lane l holds column c0 + l
+                    for (int j = 0; j < 32; ++j)
+                        x[j] = (vvalid && c0 + j < in_group) ? argmax_key(__uint_as_float(r[j]), v) : 0ull;
+                    // transposing butterfly: afterwards lane l holds column c0 + l
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) {
-                    const bool upper = (lane & o) != 0;
+                    for (int o = 16; o >= 1; o >>= 1) {
+                        const bool upper = (lane & o) != 0;
 #pragma unroll
-                    for (int i = 0; i < o; ++i) {
-                        const unsigned long long send = upper ? x[i] : x[i + o];
-                        const unsigned long long keep = upper ? x[i + o] : x[i];
-                        x[i] = umax64(keep, __shfl_xor_sync(0xffffffffu, send, o));
+                        for (int i = 0; i < o; ++i) {
+                            const unsigned long long send = upper ? x[i] : x[i + o];
+                            const unsigned long long keep = upper ? x[i + o] : x[i];
+                            x[i] = umax64(keep, __shfl_xor_sync(0xffffffffu, send, o));
+                        }
                     }
+                    red[ew][c0 + lane] = tile == 0 ? x[0] : umax64(red[ew][c0 + lane], x[0]);
                 }
-                red[ew][c0 + lane] = x[0];
             }
             tc_fence_before();
             __syncwarp();
@@ -843,29 +868,31 @@ cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int 
         e = launch_pdl_cluster(lmhead_argmax_pair_kernel, dim3((unsigned)(2 * pairs)), dim3(kLmThreads), pair_smem,
                                st, 2, tmW, tmW16, tmH, p);
     } else {
-        p.stage_bytes = kStageA + (uint32_t)p.group_nodes * 128;
+        // two W tiles per unit when both accumulators of a buffer fit in its
+        // 256 TMEM columns (up to 128 nodes)
+        p.tiles = p.group_nodes <= kTileM ? 2 : 1;
+        p.stage_bytes = (uint32_t)p.tiles * kStageA + (uint32_t)p.group_nodes * 128;
         p.stages = kSmemBudget / (int)p.stage_bytes;
         if (p.stages > kMaxStages) p.stages = kMaxStages;
         const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
-        // vocabulary units of whole 16-row boxes, at most 8 per unit, as many
+        // vocabulary units of whole 16-row boxes, at most 8 per tile, as many
         // units per SM as that needs
+        const long long max_boxes = (long long)p.tiles * (kTileM / kBoxRowsW);
         const long long boxes = ((long long)V + kBoxRowsW - 1) / kBoxRowsW;
-        const long long per_sm = (boxes + 8LL * sms - 1) / (8LL * sms);
+        const long long per_sm = (boxes + max_boxes * sms - 1) / (max_boxes * sms);
         long long units = per_sm * sms;
         if (units > boxes) units = boxes;
         if (units * p.ngroups > 0x7fffffffLL) return cudaErrorInvalidValue;
         p.units = (int)units;
         p.unit_b = (int)(boxes / units);
         p.unit_rem = (int)(boxes - (long long)p.unit_b * units);
-        const int big_rows = (p.unit_b + 1 < kTileM / kBoxRowsW ? p.unit_b + 1 : kTileM / kBoxRowsW) * kBoxRowsW;
-        CUtensorMap tmWbig, tmWsmall;
-        if (!encode_tensor_map_2d(&tmWbig, w, (uint64_t)d, (uint64_t)V, (uint64_t)d * 2, kKChunk, big_rows))
-            return cudaErrorInvalidValue;
-        if (!encode_tensor_map_2d(&tmWsmall, w, (uint64_t)d, (uint64_t)V, (uint64_t)d * 2, kKChunk,
-                                  p.unit_b * kBoxRowsW))
-            return cudaErrorInvalidValue;
+        LmWMaps maps;
+        for (int i = 0; i < kTileM / kBoxRowsW; ++i)
+            if (!encode_tensor_map_2d(&maps.m[i], w, (uint64_t)d, (uint64_t)V, (uint64_t)d * 2, kKChunk,
+                                      (i + 1) * kBoxRowsW))
+                return cudaErrorInvalidValue;
         e = launch_pdl(lmhead_argmax_tc_kernel, dim3((unsigned)(units * p.ngroups)), dim3(kLmThreads), smem, st,
-                       tmWbig, tmWsmall, tmH, p);
+                       maps, tmH, p);
     }
     count_launches(1);
     return e;
