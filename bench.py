@@ -3,7 +3,8 @@
 
 A step is one pass of the whole hot path over one batch of synthetic input:
 tree attention, LM head + argmax, accept walk and KV compaction, i.e. the
-four calls of ``include/jsv.h`` on one stream.  Inputs are resident in HBM
+calls of ``include/jsv.h`` on one stream (the walk and the compaction as the
+one fused ``jsv_accept_compact`` launch).  Inputs are resident in HBM
 when the timed region starts; L2 is flushed (a 512 MB write) before every
 timed step, outside its events.  The headline times whole steps with CUDA
 events on the launching stream; a second timed pass of the same steps puts
@@ -61,7 +62,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
-    ap.add_argument("--profile", choices=["attention", "lmhead", "accept", "compact", "tree", "qkv"],
+    ap.add_argument("--profile", choices=["attention", "lmhead", "accept", "compact", "accept_compact", "tree", "qkv"],
                     help="run only this call K times after W warm-up (for ncu); prints its mean time")
     return ap.parse_args()
 
@@ -383,7 +384,7 @@ def run_gpu(args, rank, world, local_rank):
 
     # timed region 2: the same steps with an event between calls, for the
     # per-call durations (the dominant kernel's roofline uses these)
-    evc = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    evc = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     torch.cuda.synchronize()
     for i in range(K):
         flush.fill_(i & 0xFF)
@@ -393,12 +394,10 @@ def run_gpu(args, rank, world, local_rank):
         e[1].record(stream)
         st.lmhead()
         e[2].record(stream)
-        st.accept()
+        st.accept_compact()
         e[3].record(stream)
-        st.compact()
-        e[4].record(stream)
     torch.cuda.synchronize()
-    per = np.array([[evc[i][j].elapsed_time(evc[i][j + 1]) for j in range(4)] for i in range(K)])
+    per = np.array([[evc[i][j].elapsed_time(evc[i][j + 1]) for j in range(3)] for i in range(K)])
     call_ms = per.mean(axis=0)
     assert int(st.status.item()) == 0
 
@@ -483,7 +482,7 @@ def run_gpu(args, rank, world, local_rank):
         return
 
     hbm, tf_burst, tf_sus, peak_kind = peaks()
-    names = ["attention", "lmhead", "accept", "compact"]
+    names = ["attention", "lmhead", "accept_compact"]
     share = {n: float(call_ms[j] / call_ms.sum()) for j, n in enumerate(names)}
     dom = "lmhead" if call_ms[1] >= call_ms[0] else "attention"
     dom_ms = float(call_ms[names.index(dom)])

@@ -18,6 +18,8 @@
  *   jsv_kv_compact      move the accepted path's K/V rows to contiguous
  *                       slots P..P+a of each request (ragged batches)
  *
+ * jsv_accept_compact does the last two in one launch.
+ *
  * Conventions for every call
  *   - Pointers marked "device" are CUDA device (or managed) memory; the
  *     caller allocates and owns every buffer, workspace included.  The
@@ -239,6 +241,22 @@ JSV_API jsv_status jsv_accept_path(const jsv_batch *batch, const int32_t *tokens
 JSV_API jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uint16_t *v_cache,
                           const int32_t *path, int32_t max_path, const int32_t *accept_len,
                           int32_t *new_len, void *stream);
+
+/*
+ * jsv_accept_path followed by jsv_kv_compact, in one kernel launch: the
+ * step's two latency-bound tail calls fused (the pages have no counterpart;
+ * a deployment form of the same two operations).  Every output -- path,
+ * accept_len, bonus, the K/V caches and new_len -- and every device-side
+ * error equals what the two calls in sequence produce on the same inputs.
+ * Arguments follow those two calls: the tree arrays and argmax are read, the
+ * path row is written with stride max_path, and the caches are updated in
+ * place.
+ */
+JSV_API jsv_status jsv_accept_compact(const jsv_batch *batch, const int32_t *tokens,
+                                      const int32_t *argmax, int32_t max_path,
+                                      int32_t *path, int32_t *accept_len, int32_t *bonus,
+                                      uint16_t *k_cache, uint16_t *v_cache, int32_t *new_len,
+                                      void *stream);
 
 /*
  * LM head fused with top-1 argmax for callers that cannot allocate device

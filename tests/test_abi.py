@@ -64,6 +64,8 @@ def test_host_validation_rejects_batches(lib, kw, code):
     assert st == code
     st = lib.jsv_kv_compact(ctypes.byref(b), 16, 16, 16, 8, 16, 16, None)
     assert st == code
+    st = lib.jsv_accept_compact(ctypes.byref(b), 16, 16, 8, 16, 16, 16, 16, 16, 16, None)
+    assert st == code
 
 
 def test_host_validation_other_arguments(lib):
@@ -75,6 +77,8 @@ def test_host_validation_other_arguments(lib):
     assert lib.jsv_tree_attention(ctypes.byref(b), 16, 16, 16, 0.1, 16, 256, 1, None) == 1
     assert lib.jsv_tree_attention_workspace_size(ctypes.byref(b)) > 0
     assert lib.jsv_accept_path(ctypes.byref(b), 16, 16, 0, 16, 16, 16, None) == 1
+    assert lib.jsv_accept_compact(ctypes.byref(b), 16, 16, 0, 16, 16, 16, 16, 16, 16, None) == 1
+    assert lib.jsv_accept_compact(ctypes.byref(b), 16, 16, 8, 16, 16, 16, 18, 16, 16, None) == 1
     # LM head: d not a multiple of 64, missing workspace, NULL output
     assert lib.jsv_lmhead_argmax(16, 16, 4, 100, 50, 16, None, 16, 1 << 20, None) == 2
     assert lib.jsv_lmhead_argmax(16, 16, 4, 128, 50, 16, None, None, 0, None) == 1

@@ -148,25 +148,33 @@ def test_lmhead_ties_take_smallest_index():
     assert arg.cpu().tolist() == [17, 17, 17]
 
 
-def _walk_and_compact(parents, pre, tokens, argmax, max_path=None):
+def _walk_and_compact(parents, pre, tokens, argmax, max_path=None, fused=False, mutate=None):
+    """The accept walk and the KV compaction, as two calls or as the fused
+    jsv_accept_compact; `mutate` edits the case (to plant an input error)."""
     case = small_case(parents, pre, Hq=2, Hkv=2, D=64, seed=3)
+    if mutate:
+        mutate(case)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     batch, keep = _batch(case, status)
     B = len(parents)
     mp = max_path or max(len(p) for p in parents)
     path = torch.full((B, mp), 77, dtype=torch.int32, device="cuda")
-    acc = torch.empty(B, dtype=torch.int32, device="cuda")
-    bonus = torch.empty(B, dtype=torch.int32, device="cuda")
-    nl = torch.empty(B, dtype=torch.int32, device="cuda")
+    acc = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+    bonus = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+    nl = torch.full((B,), -7, dtype=torch.int32, device="cuda")
     k, v = _dev_bf16(case["k_cache"]), _dev_bf16(case["v_cache"])
-    jsv.jsv_accept_path(batch, _dev_i32(tokens), _dev_i32(argmax), mp, path, acc, bonus)
-    jsv.jsv_kv_compact(batch, k, v, path, mp, acc, nl)
+    if fused:
+        jsv.jsv_accept_compact(batch, _dev_i32(tokens), _dev_i32(argmax), mp, path, acc, bonus, k, v, nl)
+    else:
+        jsv.jsv_accept_path(batch, _dev_i32(tokens), _dev_i32(argmax), mp, path, acc, bonus)
+        jsv.jsv_kv_compact(batch, k, v, path, mp, acc, nl)
     torch.cuda.synchronize()
     return case, dict(path=path.cpu().numpy(), acc=acc.cpu().numpy(), bonus=bonus.cpu().numpy(),
                       new_len=nl.cpu().numpy(), k=_bits(k), v=_bits(v), status=int(status.item()))
 
 
-def test_walk_and_compaction_random_batches():
+@pytest.mark.parametrize("fused", [False, True])
+def test_walk_and_compaction_random_batches(fused):
     rng = np.random.default_rng(9)
     for trial in range(6):
         B = int(rng.integers(1, 9))
@@ -180,7 +188,7 @@ def test_walk_and_compaction_random_batches():
             for c in range(1, len(p)):
                 if rng.random() < 0.8:
                     tokens[offs[b] + c] = argmax[offs[b] + p[c]]
-        case, got = _walk_and_compact(parents, pre, tokens, argmax)
+        case, got = _walk_and_compact(parents, pre, tokens, argmax, fused=fused)
         assert got["status"] == 0
         ref = oracle.accept_batch(offs, np.concatenate(parents), tokens, argmax)
         kref, vref = case["k_cache"].copy(), case["v_cache"].copy()
@@ -192,28 +200,63 @@ def test_walk_and_compaction_random_batches():
         assert np.array_equal(got["k"], kref) and np.array_equal(got["v"], vref)
 
 
-def test_full_depth_chain_and_zero_accept():
+@pytest.mark.parametrize("fused", [False, True])
+def test_full_depth_chain_and_zero_accept(fused):
     n = 300
     chain = np.arange(-1, n - 1)
     argmax = np.arange(n) + 1000
     tokens = np.concatenate([[5], argmax[:-1]])                 # everything matches
     case, got = _walk_and_compact([chain, np.array([-1, 0, 0])], [33, 7],
                                   np.concatenate([tokens, [1, 2, 3]]),
-                                  np.concatenate([argmax, [9, 9, 9]]))
+                                  np.concatenate([argmax, [9, 9, 9]]), fused=fused)
     assert got["status"] == 0
     assert got["acc"].tolist() == [n - 1, 0]
     assert got["path"][0].tolist() == list(range(n))
     assert got["new_len"].tolist() == [33 + n, 8]
 
 
-def test_path_longer_than_max_path_is_reported():
+@pytest.mark.parametrize("fused", [False, True])
+def test_path_longer_than_max_path_is_reported(fused):
     n = 10
     chain = np.arange(-1, n - 1)
     argmax = np.arange(n) + 50
     tokens = np.concatenate([[0], argmax[:-1]])
-    case, got = _walk_and_compact([chain], [3], tokens, argmax, max_path=4)
+    case, got = _walk_and_compact([chain], [3], tokens, argmax, max_path=4, fused=fused)
     assert got["status"] == jsv.JSV_ERR_DEVICE_INPUT
     assert got["path"][0].tolist() == [0, 1, 2, 3]
+
+
+def _bad_parent(case):
+    case["parent"] = case["parent"].copy()
+    case["parent"][2] = 5                      # parent index above the node's own
+
+
+def _bad_tree_page(case):
+    case["page_table"] = case["page_table"].copy()
+    case["page_table"][0, case["prefix_len"][0] // 16] = case["num_pages"] + 3
+
+
+@pytest.mark.parametrize("mutate,max_path", [(None, 4), (_bad_parent, None), (_bad_tree_page, None)])
+def test_fused_accept_compact_equals_the_two_calls(mutate, max_path):
+    """Bit-for-bit the same outputs and status as jsv_accept_path +
+    jsv_kv_compact, on a good batch cut by max_path and on inputs that the
+    device rejects (a malformed parent array, an unmapped tree page)."""
+    rng = np.random.default_rng(21)
+    parents = [synth.tiny_tree(rng, 30, 8, 2), np.arange(-1, 12), synth.tiny_tree(rng, 50, 10, 3)]
+    pre = [37, 16, 5]
+    T = sum(len(p) for p in parents)
+    argmax = rng.integers(0, 4, T)
+    tokens = rng.integers(0, 4, T)
+    offs = np.concatenate([[0], np.cumsum([len(p) for p in parents])])
+    for b, p in enumerate(parents):
+        for c in range(1, len(p)):
+            if rng.random() < 0.85:
+                tokens[offs[b] + c] = argmax[offs[b] + p[c]]
+    _, two = _walk_and_compact(parents, pre, tokens, argmax, max_path=max_path, mutate=mutate)
+    _, one = _walk_and_compact(parents, pre, tokens, argmax, max_path=max_path, mutate=mutate, fused=True)
+    assert two["status"] == jsv.JSV_ERR_DEVICE_INPUT
+    for key in two:
+        assert np.array_equal(np.asarray(one[key]), np.asarray(two[key])), key
 
 
 def test_malformed_parent_is_reported_not_trapped():

@@ -1,18 +1,9 @@
-// Greedy accept walk: one warp per request.
-//
-// JetSpec README, "JetSpec / Overview": the accepted path is chosen by the
-// target's own logits, so decoding is lossless.  At temperature 0 that is
-// the greedy descent: from the root, step to the smallest-index child whose
-// draft token equals the target's argmax at the current node, until no
-// child matches.  Children have larger indices than their parent
-// (topological order), so each step scans indices > cur with a warp ballot
-// and takes the lowest set lane of the first chunk that has a match.
-#include "jsv_internal.cuh"
+// Greedy accept walk: one warp per request (the walk itself is in walk.cuh).
+#include "walk.cuh"
 
 namespace jsv {
 
 constexpr int kWalkWarps = 4;
-constexpr int kWalkMaxNodes = 512;
 
 __global__ void __launch_bounds__(kWalkWarps * 32)
 accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
@@ -53,29 +44,14 @@ accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
     }
     __syncwarp();
 
-    int cur = 0, len = 1;
-    while (true) {
-        const int want = s_arg[w][cur];
-        int found = -1;
-        for (int j0 = cur + 1; j0 < r.n; j0 += 32) {
-            const int j = j0 + lane;
-            const bool m = j < r.n && s_par[w][j] == cur && s_tok[w][j] == want;
-            const unsigned bal = __ballot_sync(0xffffffffu, m);
-            if (bal) { found = j0 + __ffs(bal) - 1; break; }
-        }
-        if (found < 0) break;
-        if (len >= max_path) {
-            if (lane == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
-            break;
-        }
-        if (lane == 0) row[len] = found;
-        ++len;
-        cur = found;
-    }
+    int last = 0;
+    bool cut = false;
+    const int len = greedy_walk_warp(s_par[w], s_tok[w], s_arg[w], r.n, max_path, row, lane, last, cut);
+    if (cut && lane == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
     if (lane == 0) {
         row[0] = 0;
         accept_len[b] = len - 1;
-        bonus[b] = s_arg[w][cur];
+        bonus[b] = s_arg[w][last];
     }
     for (int k = len + lane; k < max_path; k += 32) row[k] = -1;
 }

@@ -110,6 +110,18 @@ jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uint16_t *v
                                             accept_len, new_len, static_cast<cudaStream_t>(stream)));
 }
 
+jsv_status jsv_accept_compact(const jsv_batch *batch, const int32_t *tokens, const int32_t *argmax,
+                              int32_t max_path, int32_t *path, int32_t *accept_len, int32_t *bonus,
+                              uint16_t *k_cache, uint16_t *v_cache, int32_t *new_len, void *stream) {
+    jsv_status s = check_batch(batch);
+    if (s != JSV_OK) return s;
+    if (!tokens || !argmax || !path || !accept_len || !bonus || !k_cache || !v_cache || !new_len || max_path < 1)
+        return JSV_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return JSV_ERR_INVALID_ARG;
+    return from_cuda(jsv::launch_accept_compact(jsv::to_args(batch), tokens, argmax, max_path, path, accept_len,
+                                                bonus, k_cache, v_cache, new_len, static_cast<cudaStream_t>(stream)));
+}
+
 jsv_status jsv_tree_qkv_rope(const jsv_batch *batch, const uint16_t *x, const uint16_t *w_qkv, int32_t d,
                              const float *rope_cos, const float *rope_sin, int32_t max_pos, uint16_t *q,
                              uint16_t *k_cache, uint16_t *v_cache, void *stream) {

@@ -155,6 +155,9 @@ cudaError_t launch_accept_path(const BatchArgs &a, const int32_t *tokens, const 
 cudaError_t launch_kv_compact(const BatchArgs &a, uint16_t *k_cache, uint16_t *v_cache,
                               const int32_t *path, int max_path, const int32_t *accept_len,
                               int32_t *new_len, cudaStream_t st);
+cudaError_t launch_accept_compact(const BatchArgs &a, const int32_t *tokens, const int32_t *argmax, int max_path,
+                                  int32_t *path, int32_t *accept_len, int32_t *bonus, uint16_t *k_cache,
+                                  uint16_t *v_cache, int32_t *new_len, cudaStream_t st);
 size_t lmhead_workspace_bytes(int T, int d, int V);
 cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int T, int d, int V,
                                  int32_t *argmax, float *max_logit, void *ws, cudaStream_t st);

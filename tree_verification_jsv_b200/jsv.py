@@ -24,7 +24,7 @@ EXPORTS = ("jsv_tree_attention_workspace_size", "jsv_tree_attention",
            "jsv_lmhead_argmax_workspace_size", "jsv_lmhead_argmax", "jsv_accept_path",
            "jsv_kv_compact", "jsv_status_string", "jsv_version", "jsv_kernel_launches",
            "jsv_lmhead_argmax_noalloc", "jsv_last_error_string", "jsv_selftest_wait_timeout",
-           "jsv_accum_logp_tree", "jsv_tree_qkv_rope")
+           "jsv_accum_logp_tree", "jsv_tree_qkv_rope", "jsv_accept_compact")
 
 # Largest node count jsv_lmhead_argmax_noalloc accepts (JSV_NOALLOC_MAX_NODES).
 NOALLOC_MAX_NODES = 8192
@@ -76,6 +76,8 @@ def load() -> ctypes.CDLL:
     lib.jsv_accept_path.restype = ctypes.c_int
     lib.jsv_kv_compact.argtypes = [bp, vp, vp, vp, i32, vp, vp, vp]
     lib.jsv_kv_compact.restype = ctypes.c_int
+    lib.jsv_accept_compact.argtypes = [bp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp]
+    lib.jsv_accept_compact.restype = ctypes.c_int
     lib.jsv_status_string.argtypes = [ctypes.c_int]
     lib.jsv_status_string.restype = ctypes.c_char_p
     lib.jsv_version.argtypes = []
@@ -208,3 +210,11 @@ def jsv_kv_compact(batch, k_cache, v_cache, path, max_path, accept_len, new_len,
     st = load().jsv_kv_compact(ctypes.byref(batch), _addr(k_cache), _addr(v_cache), _addr(path),
                                int(max_path), _addr(accept_len), _addr(new_len), _stream(stream))
     _check("jsv_kv_compact", st)
+
+
+def jsv_accept_compact(batch, tokens, argmax, max_path, path, accept_len, bonus, k_cache, v_cache, new_len,
+                       stream=None) -> None:
+    st = load().jsv_accept_compact(ctypes.byref(batch), _addr(tokens), _addr(argmax), int(max_path),
+                                   _addr(path), _addr(accept_len), _addr(bonus), _addr(k_cache),
+                                   _addr(v_cache), _addr(new_len), _stream(stream))
+    _check("jsv_accept_compact", st)

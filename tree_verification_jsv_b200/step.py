@@ -2,8 +2,10 @@
 
 ``VerifyStep`` owns the device buffers for a fixed geometry (torch is used
 for allocation and streams only) and issues, on one stream and with no host
-synchronisation, the four calls of ``include/jsv.h`` in order:
-tree attention, LM head + argmax, accept walk, KV compaction.
+synchronisation, the calls of ``include/jsv.h`` in order: tree attention,
+LM head + argmax, and the accept walk with the KV compaction (one launch,
+``jsv_accept_compact``; the separate ``jsv_accept_path`` and
+``jsv_kv_compact`` are kept as methods too).
 
 ``run_host`` is the end-to-end form: it copies the step's per-step inputs
 from pinned host memory, runs the step, and copies the accepted paths back.
@@ -11,7 +13,7 @@ The per-step inputs (tree arrays, tokens, q, hidden) live in one device
 arena and the outputs (paths, lengths) in another, each mirrored by one
 pinned host buffer, so each direction is a single copy.
 
-``capture`` records the four calls once into a CUDA graph (the engine the
+``capture`` records the step's calls once into a CUDA graph (the engine the
 JetSpec README describes replays CUDA graphs for wall-clock latency); every
 kernel is launched with programmatic dependent launch, so the graph keeps
 those overlapping edges.  ``replay`` launches the whole step in one call.
@@ -125,12 +127,19 @@ class VerifyStep:
         jsv.jsv_kv_compact(self.batch, self.k_cache, self.v_cache, self.path, self.max_path,
                            self.accept_len, self.new_len, stream=stream)
 
+    def accept_compact(self, stream=None):
+        """The walk and the compaction in one launch (same results as
+        ``accept`` followed by ``compact``)."""
+        jsv.jsv_accept_compact(self.batch, self.tokens, self.argmax, self.max_path, self.path,
+                               self.accept_len, self.bonus, self.k_cache, self.v_cache, self.new_len,
+                               stream=stream)
+
     def run(self, stream=None):
-        """One verify step: four launches sequences on one stream, no host sync."""
+        """One verify step on one stream, no host sync: tree attention, LM head
+        + argmax, then the accept walk fused with the KV compaction."""
         self.attention(stream)
         self.lmhead(stream)
-        self.accept(stream)
-        self.compact(stream)
+        self.accept_compact(stream)
 
     # -- CUDA graph -----------------------------------------------------------
     def capture(self):
