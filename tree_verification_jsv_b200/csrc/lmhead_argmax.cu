@@ -480,40 +480,69 @@ lmhead_argmax_tc_kernel(const __grid_constant__ LmWMaps tmW, const __grid_consta
 constexpr int kPairRows = 2 * kTileM;
 
 struct LmPairItem {
-    int row0, rows, g;     // the pair's rows [row0, row0 + rows), node group
+    int row0, rows;        // the pair's vocabulary rows [row0, row0 + rows)
+    int node0, nodes;      // its nodes [node0, node0 + nodes)
 };
 
-// Items of a pair.  One node group: a contiguous, balanced vocabulary range
-// (W is read once).  Several: items (tile, group), group fastest, dealt out
-// round-robin -- pair p takes items p, p + npairs, ... -- so at any moment
-// neighbouring pairs work on the same W tile for different node groups and
-// each tile comes from HBM once and from L2 for the other groups.
+// Items of a pair.
+// One node group (up to 256 nodes): the vocabulary is cut into 256-row
+// units; pair p takes `base` = units / npairs consecutive units (W read
+// once).  The `rem` units left over are cut by nodes into pieces of
+// piece_nodes nodes, dealt round-robin (pair p takes pieces p, p + npairs,
+// ...), so the last whole-unit round costs every pair the same and the
+// remainder adds at most a piece: a 2-SM MMA costs M = 256 rows whatever
+// the rows it holds, so a ragged remainder unit per pair would cost a whole
+// unit each.  A piece's pair still copies a full H box per CTA (rows past
+// T read as zeros) and the MMA reads its first piece_nodes / 2 rows.
+// Several node groups: items (tile, group), group fastest, dealt out
+// round-robin, so at any moment neighbouring pairs work on the same W tile
+// for different node groups and each tile comes from HBM once and from L2
+// for the other groups.
 struct LmPairWork {
-    int r0, r1, pair, npairs, items;
+    int pair, npairs, items;
+    int base, rem, piece_nodes, blocks;     // one node group
     __device__ LmPairWork(const LmParams &p, int pair_, int npairs_) : pair(pair_), npairs(npairs_) {
+        const int units = (p.V + kPairRows - 1) / kPairRows;
         if (p.ngroups == 1) {
-            r0 = (int)((long long)p.V * pair / npairs);
-            r1 = (int)((long long)p.V * (pair + 1) / npairs);
-            items = (r1 - r0 + kPairRows - 1) / kPairRows;
+            base = units / npairs;
+            rem = units - base * npairs;
+            const int node_blocks = (p.T + 15) / 16;
+            // pieces of whole 16-node blocks, few enough that every pair gets
+            // at most one when the remainder allows
+            piece_nodes = 16 * max(1, (node_blocks * rem + npairs - 1) / npairs);
+            blocks = (p.T + piece_nodes - 1) / piece_nodes;
+            const int pieces = rem * blocks;
+            items = base + (pair < pieces ? (pieces - pair + npairs - 1) / npairs : 0);
         } else {
-            const long long total = (long long)((p.V + kPairRows - 1) / kPairRows) * p.ngroups;
-            r0 = r1 = 0;
+            const long long total = (long long)units * p.ngroups;
+            base = rem = piece_nodes = blocks = 0;
             items = (int)((total - pair + npairs - 1) / npairs);
         }
     }
     __device__ LmPairItem item(const LmParams &p, int k) const {
         LmPairItem t;
         if (p.ngroups == 1) {
-            t.row0 = r0 + k * kPairRows;
-            t.rows = min(kPairRows, r1 - t.row0);
-            t.g = 0;
+            int unit;
+            if (k < base) {
+                unit = pair * base + k;
+                t.node0 = 0;
+                t.nodes = p.T;
+            } else {
+                const int q = pair + (k - base) * npairs;
+                unit = base * npairs + q / blocks;
+                t.node0 = (q % blocks) * piece_nodes;
+                t.nodes = min(piece_nodes, p.T - t.node0);
+            }
+            t.row0 = unit * kPairRows;
         } else {
             const long long i = pair + (long long)k * npairs;
             const int vt = (int)(i / p.ngroups);
+            const int g = (int)(i - (long long)vt * p.ngroups);
             t.row0 = vt * kPairRows;
-            t.rows = min(kPairRows, p.V - t.row0);
-            t.g = (int)(i - (long long)vt * p.ngroups);
+            t.node0 = g * p.group_nodes;
+            t.nodes = min(p.group_nodes, p.T - t.node0);
         }
+        t.rows = min(kPairRows, p.V - t.row0);
         return t;
     }
 };
@@ -585,9 +614,8 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
                 const LmPairItem t = work.item(p, it);
                 const int my_rows = pair_rows(t, rank);
                 const int my_row0 = t.row0 + rank * kTileM;
-                const int in_group = min(p.group_nodes, p.T - t.g * p.group_nodes);
-                const int nmma = (in_group + 15) & ~15;
-                const int node0 = t.g * p.group_nodes + rank * (nmma / 2);
+                const int nmma = (t.nodes + 15) & ~15;
+                const int node0 = t.node0 + rank * (nmma / 2);
                 // bytes both CTAs copy for one K-chunk (the first CTA expects them all)
                 const uint32_t tx = 2u * (uint32_t)half_nodes * 128 + w_bytes(pair_rows(t, 0)) +
                                     (pair_rows(t, 1) > 0 ? w_bytes(pair_rows(t, 1)) : 0u);
@@ -651,8 +679,7 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
                 }
                 tc_fence_after();
                 const LmPairItem t = work.item(p, it);
-                const int in_group = min(p.group_nodes, p.T - t.g * p.group_nodes);
-                const uint32_t idn = idesc_bf16_f32(kPairRows, (in_group + 15) & ~15, false, false);
+                const uint32_t idn = idesc_bf16_f32(kPairRows, (t.nodes + 15) & ~15, false, false);
                 const uint32_t d0 = tmem + (uint32_t)acc * 256u;
                 bool ok = true;
                 for (int kc = 0; kc < p.kchunks; ++kc) {
@@ -702,8 +729,8 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
             const int v0 = t.row0 + rank * kTileM;
             const int v = v0 + sub * 32 + lane;
             const bool vvalid = v < v0 + my_rows;
-            const int node0 = t.g * p.group_nodes;
-            const int in_group = min(p.group_nodes, p.T - node0);
+            const int node0 = t.node0;
+            const int in_group = t.nodes;
             const int ncols = (in_group + 31) & ~31;
             const uint32_t base = tmem + lane_addr + (uint32_t)acc * 256u;
             for (int c0 = 0; c0 < ncols; c0 += 32) {
