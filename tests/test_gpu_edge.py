@@ -92,8 +92,13 @@ def test_attention_edge_cases(name, sharp):
     attention_close(got, run_oracle_attention(case), name)
 
 
+# (64, 128, 40000): single CTAs with vocabulary units of 8 or 9 boxes, i.e.
+# units that span two 128-row W tiles; (200, 128, 38500) and (256, 64, 38500):
+# CTA pairs with more 256-row units than pairs, so the units left over are
+# split into 16-node pieces
 @pytest.mark.parametrize("T,d,V", [(1, 64, 1), (5, 128, 1000), (16, 256, 1024), (64, 512, 4099),
-                                   (130, 192, 3000), (300, 1024, 20000), (200, 256, 2500), (256, 128, 257)])
+                                   (130, 192, 3000), (300, 1024, 20000), (200, 256, 2500), (256, 128, 257),
+                                   (64, 128, 40000), (200, 128, 38500), (256, 64, 38500)])
 def test_lmhead_argmax_shapes(T, d, V):
     rng = np.random.default_rng(T * 7 + V)
     H = bf16(rng.standard_normal((T, d)) / math.sqrt(d))
