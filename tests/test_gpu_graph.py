@@ -35,3 +35,27 @@ def test_graph_replay_matches_eager_step(name):
     assert int(graphed.status.item()) == 0
     for name_ in ("out", "argmax", "max_logit", "path", "accept_len", "bonus", "new_len", "k_cache", "v_cache"):
         assert np.array_equal(_bits(getattr(eager, name_)), _bits(getattr(graphed, name_))), name_
+
+
+@pytest.mark.parametrize("name", ["tiny", "8b_64"])
+def test_host_step_matches_device_step(name):
+    """run_host (inputs copied up in two parts, the LM head on a side stream)
+    returns the same outputs as the device-resident step, over several steps
+    in a row with no synchronisation in between, and leaves the same caches."""
+    from tree_verification_jsv_b200 import build
+    from tree_verification_jsv_b200.step import VerifyStep
+    build.build()
+    wl, tokens, _ = golden_workload(name)
+    dev = VerifyStep(wl, tokens)
+    host = VerifyStep(wl, tokens)
+    outs = []
+    for _ in range(3):
+        dev.run()
+        got = host.run_host()
+        outs.append({k: v.clone() for k, v in got.items()})
+    torch.cuda.synchronize()
+    assert int(host.status.item()) == 0 and int(dev.status.item()) == 0
+    for k in ("path", "accept_len", "bonus", "new_len"):
+        assert np.array_equal(outs[-1][k].numpy(), getattr(dev, k).cpu().numpy()), k
+    for name_ in ("out", "argmax", "k_cache", "v_cache"):
+        assert np.array_equal(_bits(getattr(dev, name_)), _bits(getattr(host, name_))), name_
