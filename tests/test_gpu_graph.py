@@ -39,9 +39,9 @@ def test_graph_replay_matches_eager_step(name):
 
 @pytest.mark.parametrize("name", ["tiny", "8b_64"])
 def test_host_step_matches_device_step(name):
-    """run_host (inputs copied up in two parts, the LM head on a side stream)
-    returns the same outputs as the device-resident step, over several steps
-    in a row with no synchronisation in between, and leaves the same caches."""
+    """run_host (inputs copied up from pinned host memory, outputs copied
+    back) returns the same outputs as the device-resident step, over several
+    steps in a row, and leaves the same caches."""
     from tree_verification_jsv_b200 import build
     from tree_verification_jsv_b200.step import VerifyStep
     build.build()
@@ -52,8 +52,8 @@ def test_host_step_matches_device_step(name):
     for _ in range(3):
         dev.run()
         got = host.run_host()
+        torch.cuda.synchronize()            # the host views are filled asynchronously
         outs.append({k: v.clone() for k, v in got.items()})
-    torch.cuda.synchronize()
     assert int(host.status.item()) == 0 and int(dev.status.item()) == 0
     for k in ("path", "accept_len", "bonus", "new_len"):
         assert np.array_equal(outs[-1][k].numpy(), getattr(dev, k).cpu().numpy()), k
