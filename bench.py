@@ -212,12 +212,13 @@ def ncu_traffic(kernel_key, workload):
     p = ROOT / "profiles" / "ncu_traffic.json"
     if not p.exists():
         return None
-    d = json.loads(p.read_text()).get(kernel_key)
-    if not d or d.get("workload") != workload:
-        return None
-    if d.get("source_sha") != source_sha(*d["sources"]):
-        return None
-    return int(d["dram_bytes_per_launch"])
+    entries = json.loads(p.read_text()).get(kernel_key)
+    if isinstance(entries, dict):
+        entries = [entries]
+    for d in entries or []:
+        if d.get("workload") == workload and d.get("source_sha") == source_sha(*d["sources"]):
+            return int(d["dram_bytes_per_launch"])
+    return None
 
 
 # ---------------------------------------------------------------------------
