@@ -484,63 +484,58 @@ struct LmPairItem {
     int node0, nodes;      // its nodes [node0, node0 + nodes)
 };
 
-// Items of a pair.
-// One node group (up to 256 nodes): the vocabulary is cut into 256-row
-// units; pair p takes `base` = units / npairs consecutive units (W read
-// once).  The `rem` units left over are cut by nodes into pieces of
-// piece_nodes nodes, dealt round-robin (pair p takes pieces p, p + npairs,
-// ...), so the last whole-unit round costs every pair the same and the
-// remainder adds at most a piece: a 2-SM MMA costs M = 256 rows whatever
-// the rows it holds, so a ragged remainder unit per pair would cost a whole
-// unit each.  A piece's pair still copies a full H box per CTA (rows past
-// T read as zeros) and the MMA reads its first piece_nodes / 2 rows.
-// Several node groups: items (tile, group), group fastest, dealt out
-// round-robin, so at any moment neighbouring pairs work on the same W tile
-// for different node groups and each tile comes from HBM once and from L2
-// for the other groups.
+// Items of a pair.  An item is one 256-row vocabulary unit x one node group
+// (group fastest): with several groups, consecutive items share a W unit, so
+// at any moment neighbouring pairs read the same unit and it comes from HBM
+// once and from L2 for the other groups; with one group W is read once.
+// The `base` = items / npairs whole rounds are dealt round-robin (pair p takes
+// items p, p + npairs, ...).  The `rem` items left over would leave most pairs
+// idle for a last round -- a 2-SM MMA costs M = 256 rows and N = the group's
+// nodes whatever the rows it holds -- so they are cut by nodes into pieces of
+// piece_nodes nodes (16-node blocks, sized so that there are about as many
+// pieces as pairs), also dealt round-robin.  A piece's pair still copies a
+// full H box per CTA (rows past T read as zeros); its MMA reads the first
+// piece_nodes / 2 rows of each.
 struct LmPairWork {
     int pair, npairs, items;
-    int base, rem, piece_nodes, blocks;     // one node group
+    int base, rem, piece_nodes, pieces;
+    __device__ __forceinline__ void item_geometry(const LmParams &p, int i, int &row0, int &node0, int &nodes) const {
+        const int vt = i / p.ngroups, g = i - vt * p.ngroups;
+        row0 = vt * kPairRows;
+        node0 = g * p.group_nodes;
+        nodes = min(p.group_nodes, p.T - node0);
+    }
     __device__ LmPairWork(const LmParams &p, int pair_, int npairs_) : pair(pair_), npairs(npairs_) {
-        const int units = (p.V + kPairRows - 1) / kPairRows;
-        if (p.ngroups == 1) {
-            base = units / npairs;
-            rem = units - base * npairs;
-            const int node_blocks = (p.T + 15) / 16;
-            // pieces of whole 16-node blocks, few enough that every pair gets
-            // at most one when the remainder allows
-            piece_nodes = 16 * max(1, (node_blocks * rem + npairs - 1) / npairs);
-            blocks = (p.T + piece_nodes - 1) / piece_nodes;
-            const int pieces = rem * blocks;
-            items = base + (pair < pieces ? (pieces - pair + npairs - 1) / npairs : 0);
-        } else {
-            const long long total = (long long)units * p.ngroups;
-            base = rem = piece_nodes = blocks = 0;
-            items = (int)((total - pair + npairs - 1) / npairs);
+        const int total = ((p.V + kPairRows - 1) / kPairRows) * p.ngroups;
+        base = total / npairs;
+        rem = total - base * npairs;
+        const int group_blocks = (p.group_nodes + 15) / 16;
+        piece_nodes = 16 * max(1, (group_blocks * rem + npairs - 1) / npairs);
+        pieces = 0;
+        for (int r = 0; r < rem; ++r) {
+            int row0, node0, nodes;
+            item_geometry(p, base * npairs + r, row0, node0, nodes);
+            pieces += (nodes + piece_nodes - 1) / piece_nodes;
         }
+        items = base + (pair < pieces ? (pieces - pair + npairs - 1) / npairs : 0);
     }
     __device__ LmPairItem item(const LmParams &p, int k) const {
         LmPairItem t;
-        if (p.ngroups == 1) {
-            int unit;
-            if (k < base) {
-                unit = pair * base + k;
-                t.node0 = 0;
-                t.nodes = p.T;
-            } else {
-                const int q = pair + (k - base) * npairs;
-                unit = base * npairs + q / blocks;
-                t.node0 = (q % blocks) * piece_nodes;
-                t.nodes = min(piece_nodes, p.T - t.node0);
-            }
-            t.row0 = unit * kPairRows;
+        if (k < base) {
+            item_geometry(p, pair + k * npairs, t.row0, t.node0, t.nodes);
         } else {
-            const long long i = pair + (long long)k * npairs;
-            const int vt = (int)(i / p.ngroups);
-            const int g = (int)(i - (long long)vt * p.ngroups);
-            t.row0 = vt * kPairRows;
-            t.node0 = g * p.group_nodes;
-            t.nodes = min(p.group_nodes, p.T - t.node0);
+            // piece q: find its leftover item by walking the items' piece counts
+            int q = pair + (k - base) * npairs;
+            int r = 0, row0 = 0, node0 = 0, nodes = 0;
+            for (; r < rem; ++r) {
+                item_geometry(p, base * npairs + r, row0, node0, nodes);
+                const int nb = (nodes + piece_nodes - 1) / piece_nodes;
+                if (q < nb) break;
+                q -= nb;
+            }
+            t.row0 = row0;
+            t.node0 = node0 + q * piece_nodes;
+            t.nodes = min(piece_nodes, nodes - q * piece_nodes);
         }
         t.rows = min(kPairRows, p.V - t.row0);
         return t;
