@@ -43,6 +43,7 @@
 #include "sm100.cuh"
 
 #include <math.h>
+#include <type_traits>
 #include <string.h>
 
 namespace jsv {
@@ -124,6 +125,110 @@ struct AttnSmem {
 // region (rows of 128 B, 8-row atoms; chunk index XOR row % 8).
 __device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
     return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// The MMA issuer: one thread of the CTA issues every tcgen05.mma.  S of a
+// group reuses the TMEM of that group's previous P; the PV that reads it was
+// issued earlier and MMAs run in issue order.
+//
+// Instantiated per group count so that every TMEM address and descriptor
+// offset is a compile-time constant added to a base formed once: this
+// thread's instruction stream between two MMAs is on the tensor pipe's
+// critical path (with the group index and the addresses computed at run time
+// the MMAs issued about 1.3x slower).  A descriptor's start-address field
+// holds (address >> 4) in 14 bits; shared memory ends below 256 KB, so adding
+// an offset to a base descriptor never carries out of the field.
+template <int D, int NG>
+__device__ __forceinline__ void attention_mma_loop(uint32_t tmem, uint32_t aQ, uint32_t aKV, int ntiles,
+                                                   uint64_t *k_full, uint64_t *v_full, uint64_t *k_empty,
+                                                   uint64_t *v_empty, uint64_t *s_full, uint64_t *p_full,
+                                                   uint64_t *o_done, uint64_t *q_ready, uint64_t *drain_bar,
+                                                   volatile int *abort_sh, int32_t *dev_status) {
+    using L = AttnSmem<D>;
+    constexpr uint32_t id_s = idesc_bf16_f32(128, kKeyTile, false, false);
+    constexpr uint32_t id_o = idesc_bf16_f32(128, D, false, true);
+    constexpr uint32_t kStageStep = L::kStageBytes >> 4;           // descriptor step between K/V stages
+    uint64_t dQ = desc_kmajor_sw128(aQ);
+    uint64_t dK0 = desc_kmajor_sw128(aKV);
+    uint64_t dV0 = desc_mnmajor_sw128(aKV + L::kKVBytes, kKeyTile * 128, 1024);
+    // S(grp) = Q(grp) K^T over D in 16-wide K-steps; the K-major SW128
+    // operands hold 64 dims per 128-byte row, 8-row atoms 1 KB apart
+    auto issue_s = [&](auto grp_c, uint64_t dk) {
+        constexpr int grp = decltype(grp_c)::value;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = grp * L::kQGroupBytes + (kk >> 2) * (kGroupRows * 128) + (kk & 3) * 32;
+            const uint32_t offk = (kk >> 2) * (kKeyTile * 128) + (kk & 3) * 32;
+            mma_bf16_ss(tmem + grp * 128, dQ + (off >> 4), dk + (offk >> 4), id_s, kk > 0);
+        }
+        mma_commit(&s_full[grp]);
+    };
+    // O(grp) += P(grp) V: P from TMEM (8 columns per 16 keys), V MN-major
+    // (16 keys = 16 lines of 128 B; 64-dim blocks one K/V half apart)
+    auto issue_pv = [&](auto grp_c, uint64_t dv, uint32_t acc_first) {
+        constexpr int grp = decltype(grp_c)::value;
+#pragma unroll
+        for (int kk = 0; kk < kKeyTile / 16; ++kk)
+            mma_bf16_ts(tmem + 256 + grp * D, tmem + grp * 128 + kk * 8, dv + ((kk * 2048) >> 4), id_o,
+                        kk > 0 ? 1u : acc_first);
+        mma_commit(&o_done[grp]);
+    };
+    using G0 = std::integral_constant<int, 0>;
+    using G1 = std::integral_constant<int, 1>;
+    bool ok = mbar_wait(q_ready, 0, abort_sh);
+    // prologue: S of tile 0 for every group
+    if (ok) ok = mbar_wait(&k_full[0], 0, abort_sh);
+    if (ok) {
+        tc_fence_after();
+        issue_s(G0{}, dK0);
+        if constexpr (NG > 1) issue_s(G1{}, dK0);
+        mma_commit(&k_empty[0]);
+    }
+    for (int j = 0; ok && j < ntiles; ++j) {
+        // The bases pass through an empty asm each tile so that the compiler
+        // forms each descriptor with one add next to its MMA instead of
+        // hoisting all of them out of the loop: this warp runs on the few
+        // registers the control warps keep, and hoisted descriptors spill.
+        asm volatile("" : "+l"(dQ), "+l"(dK0), "+l"(dV0));
+        const int st = j % kStages;
+        const uint32_t ph = (uint32_t)((j / kStages) & 1);
+        const int stn = (j + 1) % kStages;
+        const uint32_t phn = (uint32_t)(((j + 1) / kStages) & 1);
+        const bool more = j + 1 < ntiles;
+        const uint64_t dv = dV0 + st * kStageStep, dkn = dK0 + stn * kStageStep;
+        const uint32_t acc_first = j > 0 ? 1u : 0u;
+        // group 0: its P and this tile's V; then, with a next tile, its K
+        ok = mbar_wait(&p_full[0], j & 1, abort_sh) && mbar_wait(&v_full[st], ph, abort_sh);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(G0{}, dv, acc_first);
+        if constexpr (NG == 1) mma_commit(&v_empty[st]);
+        if (more) {
+            ok = mbar_wait(&k_full[stn], phn, abort_sh);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(G0{}, dkn);
+            if constexpr (NG == 1) mma_commit(&k_empty[stn]);
+        }
+        if constexpr (NG > 1) {
+            ok = mbar_wait(&p_full[1], j & 1, abort_sh);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(G1{}, dv, acc_first);
+            mma_commit(&v_empty[st]);
+            if (more) {
+                issue_s(G1{}, dkn);
+                mma_commit(&k_empty[stn]);
+            }
+        }
+    }
+    if (!ok) {
+        *abort_sh = 1;
+        flag_error(dev_status, JSV_ERR_TIMEOUT);
+    }
+    int zero = 0;
+    mma_commit(drain_bar);
+    mbar_wait(drain_bar, 0, (volatile int *)&zero);
 }
 
 template <int D>
@@ -323,74 +428,14 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
-        // S of a group reuses the TMEM of that group's previous P; the PV that
-        // reads it was issued earlier and MMAs run in issue order.
         if (lane == 0 && ntiles > 0) {
-            const uint32_t id_s = idesc_bf16_f32(128, kKeyTile, false, false);
-            const uint32_t id_o = idesc_bf16_f32(128, D, false, true);
-            const uint32_t aQ = smem_addr(sQ);
-            bool ok = mbar_wait(&q_ready, 0, &abort_sh);
-            auto issue_s = [&](int grp, int kstage) {
-                const uint32_t aK = smem_addr(sKV + kstage * L::kStageBytes);
-                const uint32_t aQg = aQ + grp * L::kQGroupBytes;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (kGroupRows * 128) + (kk & 3) * 32;
-                    const uint32_t offk = (kk >> 2) * (kKeyTile * 128) + (kk & 3) * 32;
-                    mma_bf16_ss(tmem + grp * 128, desc_kmajor_sw128(aQg + off), desc_kmajor_sw128(aK + offk),
-                                id_s, kk > 0);
-                }
-                mma_commit(&s_full[grp]);
-            };
-            auto issue_pv = [&](int grp, int vstage, int jj) {
-                const uint32_t aV = smem_addr(sKV + vstage * L::kStageBytes + L::kKVBytes);
-#pragma unroll
-                for (int kk = 0; kk < kKeyTile / 16; ++kk) {
-                    // V is MN-major: 16 keys = 16 lines of 128 B; 64-dim blocks 16 KB apart
-                    mma_bf16_ts(tmem + 256 + grp * D, tmem + grp * 128 + kk * 8,
-                                desc_mnmajor_sw128(aV + kk * 2048, kKeyTile * 128, 1024), id_o,
-                                (jj > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(&o_done[grp]);
-            };
-            // prologue: S of tile 0 for both groups
-            if (ok) ok = mbar_wait(&k_full[0], 0, &abort_sh);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0, 0);
-                if (ngroups > 1) issue_s(1, 0);
-                mma_commit(&k_empty[0]);
-            }
-            for (int j = 0; ok && j < ntiles; ++j) {
-                const int st = j % kStages;
-                const uint32_t ph = (uint32_t)((j / kStages) & 1);
-                const int stn = (j + 1) % kStages;
-                const uint32_t phn = (uint32_t)(((j + 1) / kStages) & 1);
-                const bool more = j + 1 < ntiles;
-                for (int grp = 0; grp < ngroups; ++grp) {
-                    ok = mbar_wait(&p_full[grp], j & 1, &abort_sh) && (grp > 0 || mbar_wait(&v_full[st], ph, &abort_sh));
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(grp, st, j);
-                    if (grp == ngroups - 1) mma_commit(&v_empty[st]);
-                    if (more) {
-                        if (grp == 0) {
-                            ok = mbar_wait(&k_full[stn], phn, &abort_sh);
-                            if (!ok) break;
-                            tc_fence_after();
-                        }
-                        issue_s(grp, stn);
-                        if (grp == ngroups - 1) mma_commit(&k_empty[stn]);
-                    }
-                }
-            }
-            if (!ok) {
-                abort_sh = 1;
-                flag_error(a.dev_status, JSV_ERR_TIMEOUT);
-            }
-            int zero = 0;
-            mma_commit(&drain_bar);
-            mbar_wait(&drain_bar, 0, (volatile int *)&zero);
+            const uint32_t aQ = smem_addr(sQ), aKV = smem_addr(sKV);
+            if (ngroups > 1)
+                attention_mma_loop<D, 2>(tmem, aQ, aKV, ntiles, k_full, v_full, k_empty, v_empty, s_full, p_full,
+                                         o_done, &q_ready, &drain_bar, &abort_sh, a.dev_status);
+            else
+                attention_mma_loop<D, 1>(tmem, aQ, aKV, ntiles, k_full, v_full, k_empty, v_empty, s_full, p_full,
+                                         o_done, &q_ready, &drain_bar, &abort_sh, a.dev_status);
         }
     }
     } else {
