@@ -139,7 +139,7 @@ def workload_model(wl):
     lm_bytes = w_bytes + nodes * wl.d * 2 + nodes * 8
     lm_flops = 2 * nodes * wl.d * wl.V
     return {
-        "north_star_bytes": 2 * kv_row * prefix + w_bytes,
+        "step_hbm_bytes": 2 * kv_row * prefix + w_bytes,
         "attention": {"bytes": attn_bytes, "flops": attn_flops},
         "lmhead": {"bytes": lm_bytes, "flops": lm_flops},
         "step_flops": attn_flops + lm_flops,
@@ -523,10 +523,10 @@ def run_gpu(args, rank, world, local_rank):
                          "flush's own dirty lines are written back before the timed region",
                    "parallelism": f"replicas x{world}"},
         "step_latency_us": step_ms_max * 1e3,
-        "step_hbm_gbs": model["north_star_bytes"] / (step_ms_max * 1e-3) / 1e9,
-        "step_hbm_frac": model["north_star_bytes"] / (step_ms_max * 1e-3) / 1e9 / hbm,
+        "step_hbm_gbs": model["step_hbm_bytes"] / (step_ms_max * 1e-3) / 1e9,
+        "step_hbm_frac": model["step_hbm_bytes"] / (step_ms_max * 1e-3) / 1e9 / hbm,
         "step_tensor_frac": model["step_flops"] / (step_ms_max * 1e-3) / 1e12 / tf_burst,
-        "north_star_bytes": model["north_star_bytes"],
+        "step_hbm_bytes": model["step_hbm_bytes"],
         "call_us": {n: float(call_ms[j] * 1e3) for j, n in enumerate(names)},
         "call_share": share,
         "call_sum_us": float(call_ms.sum() * 1e3),
