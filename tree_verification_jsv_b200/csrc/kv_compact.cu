@@ -111,7 +111,6 @@ accept_compact_kernel(BatchArgs a, const int32_t *__restrict__ tokens, const int
                       int32_t *__restrict__ bonus, uint16_t *__restrict__ k_cache, uint16_t *__restrict__ v_cache,
                       int32_t *__restrict__ new_len) {
     pdl_allow_dependents();
-    pdl_wait_predecessor();
     extern __shared__ uint4 stage[];      // [kCompactChunk][heads][D/8]
     __shared__ int s_src[kCompactChunk], s_dst[kCompactChunk];
     __shared__ int32_t s_par[kWalkMaxNodes], s_tok[kWalkMaxNodes], s_arg[kWalkMaxNodes], s_path[kWalkMaxNodes];
@@ -124,9 +123,25 @@ accept_compact_kernel(BatchArgs a, const int32_t *__restrict__ tokens, const int
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int32_t *row = path + (size_t)b * max_path;
 
+    // The request's geometry and page entries are read while the previous
+    // launch (the LM head) may still run: no call of this library writes
+    // prefix_len, node_offsets or page_table.  The tree, the draft tokens and
+    // the argmax (which jsv_accum_logp_tree and the LM head write), and every
+    // write to the outputs or the caches, come after the wait (the
+    // compaction overwrites cache rows that the attention reads, and the LM
+    // head completes after the attention).
     Request r;
     const bool req_ok = load_request(a, b, r) && r.n <= kWalkMaxNodes;
-    int par_bad = 0;
+    int par_bad = 0, bad = 0;
+    if (req_ok) {
+        // every page the move touches must be mapped (the compaction's check)
+        const int pg0 = r.P / a.page_size, pg1 = (r.P + r.n - 1) / a.page_size;
+        for (int pg = pg0 + threadIdx.x; pg <= pg1; pg += blockDim.x) {
+            const int page = a.page_table[(size_t)b * a.max_pages_per_req + pg];
+            if (page < 0 || page >= a.num_pages) bad = 1;
+        }
+    }
+    pdl_wait_predecessor();
     if (req_ok) {
         for (int j = threadIdx.x; j < r.n; j += blockDim.x) {
             const int p = a.parent[r.base + j];
@@ -176,13 +191,6 @@ accept_compact_kernel(BatchArgs a, const int32_t *__restrict__ tokens, const int
     __syncthreads();
     const int acc = s_len - 1;
 
-    // every page the move touches must be mapped (the compaction's check)
-    int bad = 0;
-    const int pg0 = r.P / a.page_size, pg1 = (r.P + r.n - 1) / a.page_size;
-    for (int pg = pg0 + threadIdx.x; pg <= pg1; pg += blockDim.x) {
-        const int page = a.page_table[(size_t)b * a.max_pages_per_req + pg];
-        if (page < 0 || page >= a.num_pages) bad = 1;
-    }
     bad = __syncthreads_or(bad);
     if (bad) {
         if (threadIdx.x == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
