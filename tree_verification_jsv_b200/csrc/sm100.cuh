@@ -179,16 +179,6 @@ __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// 32 lanes x 16 consecutive columns stored from registers.
-__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-
 // 32 lanes x 32 consecutive columns stored from registers.
 __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
@@ -274,37 +264,6 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                  : "memory");
 }
 
-// Warp-collective forms of the three above: every lane of the warp executes
-// them with the same (warp-uniform) operands and one elected lane issues the
-// instruction, so descriptors stay in uniform registers.
-__device__ __forceinline__ void mma_bf16_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void mma_bf16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void mma_commit_warp(uint64_t *bar) {
-    asm volatile(
-        "{\n\t.reg .pred e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_addr(bar))
-        : "memory");
-}
-
 // ---------------------------------------------------------- CTA pairs
 // Helpers for a cluster of two CTAs sharing 2-SM tcgen05.mma (cta_group::2).
 // No load here multicasts: each CTA copies its own half of the operands.
@@ -368,28 +327,9 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
 }
 // D[tmem of both CTAs] (+)= A * B^T with M = 256: A rows 0..127 from this
 // CTA's shared memory and 128..255 from the peer's at the same offset; B's
-// N columns split in halves the same way.  Issued by one thread of the
-// first CTA of the pair.
-__device__ __forceinline__ void mma_bf16_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u)
-        : "memory");
-}
-// Arrive once on `bar` in every CTA of `cta_mask` when the pair MMAs issued so
-// far by this thread have completed.
-__device__ __forceinline__ void mma_commit_pair(uint64_t *bar, uint16_t cta_mask) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_addr(bar)),
-        "h"(cta_mask)
-        : "memory");
-}
-// Warp-collective forms: every lane executes them with warp-uniform operands
-// and one elected lane issues.
+// N columns split in halves the same way.  Warp-collective: every lane of a
+// warp of the first CTA executes it with warp-uniform operands (descriptors
+// stay in uniform registers) and one elected lane issues it.
 __device__ __forceinline__ void mma_bf16_ss_pair_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                       uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -401,6 +341,8 @@ __device__ __forceinline__ void mma_bf16_ss_pair_warp(uint32_t d_tmem, uint64_t 
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u)
         : "memory");
 }
+// Arrive once on `bar` in every CTA of `cta_mask` when the pair MMAs issued
+// so far by this warp have completed (warp-collective, one elected lane).
 __device__ __forceinline__ void mma_commit_pair_warp(uint64_t *bar, uint16_t cta_mask) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
