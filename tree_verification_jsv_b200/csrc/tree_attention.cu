@@ -197,16 +197,20 @@ __device__ __forceinline__ void attention_mma_loop(uint32_t tmem, uint32_t aQ, u
         const bool more = j + 1 < ntiles;
         const uint64_t dv = dV0 + st * kStageStep, dkn = dK0 + stn * kStageStep;
         const uint32_t acc_first = j > 0 ? 1u : 0u;
-        // group 0: its P and this tile's V; then, with a next tile, its K
-        ok = mbar_wait(&p_full[0], j & 1, abort_sh) && mbar_wait(&v_full[st], ph, abort_sh);
+        // This tile's V and the next tile's K land well before the P they
+        // pair with: wait for them first, so that no wait but P's sits
+        // between P's arrival and the MMAs it releases.  (K of tile j+1 only
+        // needs S of tile j-1 to have released its stage, and V of tile j
+        // only PV of tile j-2.)
+        ok = mbar_wait(&v_full[st], ph, abort_sh) && (!more || mbar_wait(&k_full[stn], phn, abort_sh));
+        if (!ok) break;
+        // group 0: PV of this tile, then S of the next
+        ok = mbar_wait(&p_full[0], j & 1, abort_sh);
         if (!ok) break;
         tc_fence_after();
         issue_pv(G0{}, dv, acc_first);
         if constexpr (NG == 1) mma_commit(&v_empty[st]);
         if (more) {
-            ok = mbar_wait(&k_full[stn], phn, abort_sh);
-            if (!ok) break;
-            tc_fence_after();
             issue_s(G0{}, dkn);
             if constexpr (NG == 1) mma_commit(&k_empty[stn]);
         }
