@@ -34,8 +34,10 @@
 //               O is rescaled in TMEM only when the running max grows by
 //               more than 8 (2^8), which keeps exp2 arguments bounded
 // While one group computes its softmax the tensor core runs the other
-// group's products, so neither the exp2 pipe nor the tensor pipe waits on
-// the other for long.
+// group's products.  The overlap is partial: a group's softmax (about 1,950
+// cycles a tile on B200) outlasts the other group's 16 MMAs (about 1,250), so
+// a tile takes about 3,600 cycles against 2,048 of tensor work, bound by the
+// cycle S -> softmax -> P -> PV, S of the next tile.
 // TMEM columns: S/P of group 0 [0,128), of group 1 [128,256); O of group 0
 // [256, 256+D), of group 1 [256+D, 256+2D).
 // Shared memory: Q (2 groups x 16 KB per 64 dims), 2 x (K, V) stages.
