@@ -568,7 +568,10 @@ def main():
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+        # a short timeout, so that the ranks still waiting end with an error if
+        # one rank fails (tests/test_multirank.py shows it with gloo); it is
+        # well above the longest stretch between two collectives here
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     try:
         run_gpu(args, rank, world, local_rank)
     finally:

@@ -4,6 +4,8 @@ cross-rank aggregation is checked here on CPU with world_size 2 over gloo."""
 import os
 import socket
 import sys
+import time
+from datetime import timedelta
 from pathlib import Path
 
 import pytest
@@ -58,3 +60,50 @@ def test_single_rank_aggregation_is_identity():
     import bench
     assert bench.reduce_max_over_ranks([1.5, 2.5], device="cpu") == [1.5, 2.5]
     assert bench.whole_job_value(256, 1, 0.5) == pytest.approx(512_000.0)
+
+
+def _dying_worker(rank, world, port, queue, how):
+    """Rank 1 fails before the cross-rank reduction, between steps with
+    nothing in flight: it exits ("exit") or stops answering without leaving
+    ("stall").  Rank 0 must get an error from the reduction, at the latest
+    when the process group's timeout runs out, instead of waiting forever."""
+    sys.path.insert(0, str(ROOT))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=3))
+    if rank == 1:
+        queue.put((rank, "left"))
+        queue.close()
+        queue.join_thread()
+        if how == "stall":
+            time.sleep(10)
+        os._exit(3)
+    t0 = time.monotonic()
+    try:
+        bench.reduce_max_over_ranks([1.0], device="cpu")
+        queue.put((rank, "no error"))
+    except Exception as e:  # the backend's timeout or connection error
+        queue.put((rank, f"error after {time.monotonic() - t0:.1f}s: {type(e).__name__}"))
+    queue.close()
+    queue.join_thread()
+    os._exit(0)
+
+
+@pytest.mark.parametrize("how", ["exit", "stall"])
+def test_lost_rank_ends_the_reduction_with_an_error_gloo(how):
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    procs = [ctx.Process(target=_dying_worker, args=(r, world, port, queue, how)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = dict(queue.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+    assert results[1] == "left"
+    assert results[0].startswith("error after"), results[0]
+    waited = float(results[0].split()[2].split("s")[0])
+    assert waited < 60.0
+    assert procs[0].exitcode == 0 and procs[1].exitcode == 3
