@@ -193,8 +193,13 @@ JSV_API size_t jsv_lmhead_argmax_workspace_size(int32_t T, int32_t d, int32_t V)
  *   workspace  device scratch of jsv_lmhead_argmax_workspace_size() bytes,
  *              8-B aligned, ZERO-FILLED before its first use (e.g. one
  *              cudaMemsetAsync when it is allocated); every call leaves it
- *              zero-filled again, so it is reused without clearing.  After a
- *              call that failed on the device, zero it again.
+ *              zero-filled again, so it is reused without clearing.
+ *   dev_status device [1] int32 or NULL.  A bounded wait of the kernel that
+ *              gave up writes JSV_ERR_TIMEOUT (compare-and-swap from 0); the
+ *              call's argmax and max_logit are then unspecified, and the
+ *              workspace is still left zero-filled (every CTA counts the work
+ *              it took, finished or abandoned, and the CTA that completes the
+ *              count clears the keys and the counter).
  * Ordering: the kernel reads `hidden` and `w` while the previous launch on
  * the stream may still be running (it waits for that launch only before it
  * touches the workspace and the outputs), so the tree-attention kernels of
@@ -207,7 +212,8 @@ JSV_API size_t jsv_lmhead_argmax_workspace_size(int32_t T, int32_t d, int32_t V)
 JSV_API jsv_status jsv_lmhead_argmax(const uint16_t *hidden, const uint16_t *w,
                              int32_t T, int32_t d, int32_t V,
                              int32_t *argmax, float *max_logit,
-                             void *workspace, size_t workspace_bytes, void *stream);
+                             void *workspace, size_t workspace_bytes,
+                             int32_t *dev_status, void *stream);
 
 /*
  * Greedy accept walk (README, "JetSpec / Overview": lossless by
@@ -250,7 +256,9 @@ JSV_API jsv_status jsv_kv_compact(const jsv_batch *batch, uint16_t *k_cache, uin
  * error equals what the two calls in sequence produce on the same inputs.
  * Arguments follow those two calls: the tree arrays and argmax are read, the
  * path row is written with stride max_path, and the caches are updated in
- * place.
+ * place.  Every argument, the batch geometry included, is read only after
+ * the previous launch on the stream has completed, so new_len of one step
+ * may be passed back as the next step's prefix_len.
  */
 JSV_API jsv_status jsv_accept_compact(const jsv_batch *batch, const int32_t *tokens,
                                       const int32_t *argmax, int32_t max_path,
@@ -267,7 +275,7 @@ JSV_API jsv_status jsv_accept_compact(const jsv_batch *batch, const int32_t *tok
  * node) is a fixed file-scope device array inside the library instead of a
  * workspace argument.  The caller still passes inputs and outputs.
  *   - T must be <= JSV_NOALLOC_MAX_NODES, else JSV_ERR_UNSUPPORTED; the
- *     other arguments follow jsv_lmhead_argmax.
+ *     other arguments, dev_status included, follow jsv_lmhead_argmax.
  *   - The array ((JSV_NOALLOC_MAX_NODES + 1) * 8 bytes) is held on every GPU
  *     that loads the library until the process exits.
  *   - The first call on a device looks up the array's device address (with
@@ -275,7 +283,8 @@ JSV_API jsv_status jsv_accept_compact(const jsv_batch *batch, const int32_t *tok
  *     stream capture.
  *   - Nothing is allocated or freed: no cudaMalloc, cudaFree or allocating
  *     library routine.  The array starts zeroed and every call leaves the
- *     keys it used zeroed again.
+ *     keys it used and the counter zeroed again, a call that reported
+ *     JSV_ERR_TIMEOUT included (its outputs are then unspecified).
  *   - Every call shares the one array, which keeps the last call's contents:
  *     calls whose kernels overlap on the GPU (different streams, or
  *     different host threads on one device) race and give wrong results.
@@ -284,7 +293,8 @@ JSV_API jsv_status jsv_accept_compact(const jsv_batch *batch, const int32_t *tok
 #define JSV_NOALLOC_MAX_NODES 8192
 JSV_API jsv_status jsv_lmhead_argmax_noalloc(const uint16_t *hidden, const uint16_t *w,
                                              int32_t T, int32_t d, int32_t V,
-                                             int32_t *argmax, float *max_logit, void *stream);
+                                             int32_t *argmax, float *max_logit,
+                                             int32_t *dev_status, void *stream);
 
 /* Number of kernels this library has launched in the calling process since
  * it was loaded (all devices, all streams).  A diagnostic for counting the
@@ -302,6 +312,26 @@ JSV_API uint64_t jsv_kernel_launches(void);
  * compare-and-swap from 0) and exits, leaving the context usable.
  */
 JSV_API jsv_status jsv_selftest_wait_timeout(int32_t *dev_status, uint32_t limit_us, void *stream);
+
+/*
+ * Failure-detection self-test of the LM head's timeout path.  Runs the LM head
+ * exactly as jsv_lmhead_argmax does with `workspace` (or, with workspace
+ * NULL, as jsv_lmhead_argmax_noalloc does, on the library's scratch array),
+ * except that the producer warp of the first CTA -- the first CTA pair for
+ * trees above 128 nodes -- first waits on a barrier that nothing signals,
+ * with the limit shortened to `limit_us` microseconds (1 .. 2,000,000).  That
+ * wait gives up before the CTA has issued any copy: the CTA writes
+ * JSV_ERR_TIMEOUT to *dev_status (device int32, required, compare-and-swap
+ * from 0), stops, and the rest of the grid completes.  argmax and max_logit
+ * are then unspecified; the workspace (or scratch array) is left zeroed, so
+ * the next ordinary call on it returns the right result.  Other arguments
+ * and checks follow jsv_lmhead_argmax (and the T limit of the no-alloc form).
+ */
+JSV_API jsv_status jsv_selftest_lmhead_timeout(const uint16_t *hidden, const uint16_t *w,
+                                               int32_t T, int32_t d, int32_t V,
+                                               int32_t *argmax, float *max_logit,
+                                               void *workspace, size_t workspace_bytes,
+                                               int32_t *dev_status, uint32_t limit_us, void *stream);
 
 /* Text of the last CUDA error behind a JSV_ERR_CUDA returned to the calling
  * host thread (a launch or runtime call that failed), or a fixed message if

@@ -127,3 +127,63 @@ def attention_close(got, want, what=""):
     assert not bad.any(), (f"{what}: {bad.sum()} elems beyond tight bound, max err {err.max()}, "
                            f"max|o| {np.abs(want).max()}")
     return float(err.max())
+
+
+def _bits_t(t):
+    import torch
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def sample_rows(wl, n, seed):
+    """Seeded (node, head) rows plus the root and the deepest node of every
+    request (first and last head)."""
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for b in range(wl.B):
+        sl = wl.request_nodes(b)
+        dep = synth.depths(wl.parent[sl])
+        for t in (sl.start, sl.start + int(np.argmax(dep))):
+            rows.add((t, 0))
+            rows.add((t, wl.Hq - 1))
+    while len(rows) < n:
+        rows.add((int(rng.integers(wl.T)), int(rng.integers(wl.Hq))))
+    return np.array(sorted(rows), dtype=np.int32)
+
+
+def assert_step_matches_oracle(st, wl, tokens, gold_arg, k0, v0, what):
+    """Every output of one verify step held by ``st`` (a VerifyStep that ran
+    once on caches k0/v0) against the oracle: argmax bit-exact against the
+    certified goldens, path / accept length / bonus / new length bit-exact,
+    the ENTIRE K and V caches bytewise, and the attention within the
+    tolerance of ``attention_close`` (all rows of small workloads, a seeded
+    sample of rows computed one by one on large ones)."""
+    import oracle
+    assert int(st.status.item()) == 0, what
+    arg = st.argmax.cpu().numpy()
+    assert np.array_equal(arg, gold_arg), f"{what}: {(arg != gold_arg).sum()} argmax mismatches"
+    ref = oracle.accept_batch(wl.node_offsets, wl.parent, tokens, gold_arg)
+    path = st.path.cpu().numpy()
+    acc = st.accept_len.cpu().numpy()
+    bonus = st.bonus.cpu().numpy()
+    for b, (p, a, bo) in enumerate(ref):
+        assert acc[b] == a and bonus[b] == bo, what
+        assert path[b, :a + 1].tolist() == p, what
+        assert np.all(path[b, a + 1:] == -1), what
+    kref, vref = k0.copy(), v0.copy()
+    new_len = oracle.kv_compact(kref, vref, wl.page_table, wl.prefix_len, [r[0] for r in ref])
+    assert np.array_equal(st.new_len.cpu().numpy(), new_len), what
+    assert np.array_equal(_bits_t(st.k_cache), kref), what
+    assert np.array_equal(_bits_t(st.v_cache), vref), what
+    # attention (computed before the compaction, on the original caches)
+    saved = wl.k_cache, wl.v_cache
+    wl.k_cache, wl.v_cache = k0, v0
+    try:
+        got_all = synth.bf16_bits_to_f32(_bits_t(st.out)).astype(np.float64)
+        if wl.T * wl.Hq <= 4096:
+            attention_close(got_all, oracle.tree_attention_wl(wl), what)
+        else:
+            rows = sample_rows(wl, 384, seed=7)
+            want = oracle.tree_attention_wl(wl, rows=rows)
+            attention_close(got_all[rows[:, 0], rows[:, 1]], want, what)
+    finally:
+        wl.k_cache, wl.v_cache = saved

@@ -80,14 +80,26 @@ def test_host_validation_other_arguments(lib):
     assert lib.jsv_accept_compact(ctypes.byref(b), 16, 16, 0, 16, 16, 16, 16, 16, 16, None) == 1
     assert lib.jsv_accept_compact(ctypes.byref(b), 16, 16, 8, 16, 16, 16, 18, 16, 16, None) == 1
     # LM head: d not a multiple of 64, missing workspace, NULL output
-    assert lib.jsv_lmhead_argmax(16, 16, 4, 100, 50, 16, None, 16, 1 << 20, None) == 2
-    assert lib.jsv_lmhead_argmax(16, 16, 4, 128, 50, 16, None, None, 0, None) == 1
-    assert lib.jsv_lmhead_argmax(16, 16, 4, 128, 50, None, None, 16, 1 << 20, None) == 1
+    assert lib.jsv_lmhead_argmax(16, 16, 4, 100, 50, 16, None, 16, 1 << 20, None, None) == 2
+    assert lib.jsv_lmhead_argmax(16, 16, 4, 128, 50, 16, None, None, 0, None, None) == 1
+    assert lib.jsv_lmhead_argmax(16, 16, 4, 128, 50, None, None, 16, 1 << 20, None, None) == 1
     assert lib.jsv_lmhead_argmax_workspace_size(4, 128, 50) >= 32
     # bounded-wait self-test: NULL status word, limits out of range
     assert lib.jsv_selftest_wait_timeout(None, 10, None) == 1
     assert lib.jsv_selftest_wait_timeout(16, 0, None) == 1
     assert lib.jsv_selftest_wait_timeout(16, 3_000_000, None) == 1
+    # LM-head timeout self-test: status word required, limit in range, the
+    # workspace or the no-alloc limit checked like the entry point it mimics
+    big = jsv.NOALLOC_MAX_NODES + 1
+    assert lib.jsv_selftest_lmhead_timeout(16, 16, 4, 128, 50, 16, None, 16, 1 << 20, None, 10, None) == 1
+    assert lib.jsv_selftest_lmhead_timeout(16, 16, 4, 128, 50, 16, None, 16, 1 << 20, 16, 0, None) == 1
+    assert lib.jsv_selftest_lmhead_timeout(16, 16, 4, 128, 50, 16, None, 16, 1, 16, 10, None) == 1
+    assert lib.jsv_selftest_lmhead_timeout(16, 16, big, 128, 50, 16, None, None, 0, 16, 10, None) == 2
+    assert lib.jsv_selftest_lmhead_timeout(16, 16, 4, 100, 50, 16, None, None, 0, 16, 10, None) == 2
+    # the no-alloc entry point: the node limit and the LM head's own checks
+    assert lib.jsv_lmhead_argmax_noalloc(16, 16, big, 128, 50, 16, None, None, None) == 2
+    assert lib.jsv_lmhead_argmax_noalloc(16, 16, 4, 100, 50, 16, None, None, None) == 2
+    assert lib.jsv_lmhead_argmax_noalloc(16, 16, 4, 128, 50, None, None, None, None) == 1
 
 
 def test_binding_raises_without_library(monkeypatch, tmp_path):

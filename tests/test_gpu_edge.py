@@ -56,7 +56,7 @@ def run_attention(case, **over):
     v = _dev_bf16(case["v_cache"])
     T = int(case["node_offsets"][-1])
     out = torch.zeros((T, case["Hq"], case["D"]), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(max(256, jsv.jsv_tree_attention_workspace_size(batch)), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(max(256, jsv.jsv_tree_attention_workspace_size(batch)), dtype=torch.uint8, device="cuda")
     jsv.jsv_tree_attention(batch, q, k, v, case["scale"], out, ws)
     torch.cuda.synchronize()
     return synth.bf16_bits_to_f32(_bits(out)).astype(np.float64), int(status.item())

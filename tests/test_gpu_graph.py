@@ -1,17 +1,46 @@
-"""The verify step captured in a CUDA graph gives the same bytes as the
-eager step (argmax, walk, compaction, attention output), on the tiny and
-the Qwen3-8B-shaped 64-node workloads."""
+"""The verify step captured in a CUDA graph: its replay matches the oracle
+(argmax, walk, compaction, attention output) on the tiny and the
+Qwen3-8B-shaped 64- and 256-node workloads, and gives the same bytes as the
+eager step; the end-to-end form through host buffers gives the device
+step's outputs."""
 import numpy as np
 import pytest
 import torch
 
-from helpers import golden_workload
+from helpers import assert_step_matches_oracle, golden_workload
 
 pytestmark = pytest.mark.gpu
 
 
 def _bits(t):
     return t.view(torch.int16).cpu().numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["tiny", "8b_64", "8b_256"])
+def test_graph_replay_matches_oracle(name):
+    """Capture, restore the caches the capture's warm-up step compacted, then
+    replay twice on the restored caches: each replay is one whole verify
+    step and must match the oracle (the second replay restores the caches
+    first, so it starts from the same state)."""
+    from tree_verification_jsv_b200 import build
+    from tree_verification_jsv_b200.step import VerifyStep
+    build.build()
+    wl, tokens, gold_arg = golden_workload(name)
+    k0, v0 = wl.k_cache.copy(), wl.v_cache.copy()
+    st = VerifyStep(wl, tokens)
+    kd, vd = st.k_cache.clone(), st.v_cache.clone()
+    st.capture()                            # runs one eager step first
+    for rep in range(2):
+        st.k_cache.copy_(kd)
+        st.v_cache.copy_(vd)
+        st.status.zero_()
+        st.out.zero_()
+        st.argmax.fill_(-1)
+        st.path.fill_(-9)
+        torch.cuda.synchronize()
+        st.replay()
+        torch.cuda.synchronize()
+        assert_step_matches_oracle(st, wl, tokens, gold_arg, k0, v0, f"{name} replay {rep}")
 
 
 @pytest.mark.parametrize("name", ["tiny", "8b_64"])

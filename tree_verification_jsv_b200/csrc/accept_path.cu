@@ -60,7 +60,7 @@ cudaError_t launch_accept_path(const BatchArgs &a, const int32_t *tokens, const 
                                int max_path, int32_t *path, int32_t *accept_len, int32_t *bonus,
                                cudaStream_t st) {
     dim3 grid((a.B + kWalkWarps - 1) / kWalkWarps);
-    static bool carve[64] = {};
+    static PerDeviceOnce carve;
     cudaError_t e = prefer_max_shared(accept_path_kernel, carve);
     if (e != cudaSuccess) return e;
     e = launch_pdl(accept_path_kernel, grid, dim3(kWalkWarps * 32), 0, st, a, tokens, argmax, max_path,

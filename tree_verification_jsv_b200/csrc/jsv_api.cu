@@ -37,6 +37,9 @@ jsv_status check_batch(const jsv_batch *b) {
     return JSV_OK;
 }
 
+}  // namespace
+
+namespace jsv {
 thread_local cudaError_t t_last_error = cudaSuccess;
 
 jsv_status from_cuda(cudaError_t e) {
@@ -45,7 +48,16 @@ jsv_status from_cuda(cudaError_t e) {
     return JSV_ERR_CUDA;
 }
 
-}  // namespace
+jsv_status check_lmhead_args(const uint16_t *hidden, const uint16_t *w, int32_t T, int32_t d, int32_t V,
+                             const int32_t *argmax) {
+    if (!hidden || !w || !argmax || T < 1 || d < 1 || V < 1) return JSV_ERR_INVALID_ARG;
+    if (d % 64 != 0 || d > 16384) return JSV_ERR_UNSUPPORTED;
+    if (!aligned(hidden, 16) || !aligned(w, 16)) return JSV_ERR_INVALID_ARG;
+    return JSV_OK;
+}
+}  // namespace jsv
+
+using jsv::from_cuda;
 
 extern "C" {
 
@@ -78,13 +90,12 @@ size_t jsv_lmhead_argmax_workspace_size(int32_t T, int32_t d, int32_t V) {
 
 jsv_status jsv_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int32_t T, int32_t d,
                              int32_t V, int32_t *argmax, float *max_logit, void *workspace,
-                             size_t workspace_bytes, void *stream) {
-    if (!hidden || !w || !argmax || T < 1 || d < 1 || V < 1) return JSV_ERR_INVALID_ARG;
-    if (d % 64 != 0 || d > 16384) return JSV_ERR_UNSUPPORTED;
-    if (!aligned(hidden, 16) || !aligned(w, 16)) return JSV_ERR_INVALID_ARG;
+                             size_t workspace_bytes, int32_t *dev_status, void *stream) {
+    jsv_status s = jsv::check_lmhead_args(hidden, w, T, d, V, argmax);
+    if (s != JSV_OK) return s;
     const size_t need = jsv::lmhead_workspace_bytes(T, d, V);
     if (workspace_bytes < need || !workspace || !aligned(workspace, 8)) return JSV_ERR_INVALID_ARG;
-    return from_cuda(jsv::launch_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, workspace,
+    return from_cuda(jsv::launch_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, workspace, dev_status, 0,
                                                static_cast<cudaStream_t>(stream)));
 }
 
@@ -165,8 +176,8 @@ int32_t jsv_version(void) { return 100; }
 
 const char *jsv_last_error_string(void) {
     static thread_local char buf[512];
-    if (t_last_error == cudaSuccess) return "no CUDA error recorded";
-    snprintf(buf, sizeof buf, "%s%s%s", cudaGetErrorString(t_last_error), jsv::t_launch_note[0] ? " -- " : "",
+    if (jsv::t_last_error == cudaSuccess) return "no CUDA error recorded";
+    snprintf(buf, sizeof buf, "%s%s%s", cudaGetErrorString(jsv::t_last_error), jsv::t_launch_note[0] ? " -- " : "",
              jsv::t_launch_note);
     return buf;
 }

@@ -5,6 +5,9 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/jsv.h"
 
 namespace jsv {
@@ -26,23 +29,46 @@ inline BatchArgs to_args(const jsv_batch *b) {
     return a;
 }
 
+// One-time host set-up per device (kernel attributes): the first call made
+// with a device current runs it under a lock, later calls read a flag, so
+// host threads that make their first calls at the same time do not race.  A
+// set-up that failed is not recorded and runs again on the next call.
+// Devices past the table run it on every call.
+class PerDeviceOnce {
+public:
+    template <typename F>
+    cudaError_t run(F &&f) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kDevices) return f();
+        if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+        e = f();
+        if (e == cudaSuccess) done_[dev].store(true, std::memory_order_release);
+        return e;
+    }
+
+private:
+    static constexpr int kDevices = 64;
+    std::atomic<bool> done_[kDevices] = {};
+    std::mutex mu_;
+};
+
 // Kernels of a step run side by side on one SM (programmatic dependent
 // launch lets the next kernel start early), but an SM's split between L1 and
 // shared memory stays fixed while any CTA is resident on it.  A small kernel
 // left to the driver's default split would take a large L1 and keep the
 // LM-head and attention CTAs, which need most of the shared memory, off every
 // SM it occupies until it exits.  So every kernel asks for the largest shared
-// carveout; `done` is the call site's once-per-device flag array.
+// carveout, once per device.
 template <typename K>
-inline cudaError_t prefer_max_shared(K *kernel, bool (&done)[64]) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || done[dev]) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared);
-    if (e == cudaSuccess) done[dev] = true;
-    return e;
+inline cudaError_t prefer_max_shared(K *kernel, PerDeviceOnce &once) {
+    return once.run([&]() {
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    (int)cudaSharedmemCarveoutMaxShared);
+    });
 }
 
 // Programmatic dependent launch: every kernel of the library is launched so
@@ -102,6 +128,17 @@ __device__ __forceinline__ long long slot_phys_row(const BatchArgs &a, int b, in
 // Count of kernel launches issued by the library (see jsv_kernel_launches).
 void count_launches(int n);
 
+// Host-side status of a CUDA call (records the error for jsv_last_error_string).
+jsv_status from_cuda(cudaError_t e);
+
+// Host-side checks shared by the LM-head entry points.
+jsv_status check_lmhead_args(const uint16_t *hidden, const uint16_t *w, int32_t T, int32_t d, int32_t V,
+                             const int32_t *argmax);
+
+// Device address of the allocation-free LM head's scratch array on the
+// current device (looked up with that device current on first use).
+cudaError_t noalloc_scratch(void **out);
+
 // Record the resources of a kernel whose launch failed, for
 // jsv_last_error_string (thread-local).
 void note_launch_failure(const char *what, int regs, int max_threads, size_t static_smem, int max_dyn_smem,
@@ -159,8 +196,11 @@ cudaError_t launch_accept_compact(const BatchArgs &a, const int32_t *tokens, con
                                   int32_t *path, int32_t *accept_len, int32_t *bonus, uint16_t *k_cache,
                                   uint16_t *v_cache, int32_t *new_len, cudaStream_t st);
 size_t lmhead_workspace_bytes(int T, int d, int V);
+// status: device status word or NULL; inject_ns: 0, or the limit of the
+// failure-detection self-test's injected wait (jsv_selftest_lmhead_timeout)
 cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int T, int d, int V,
-                                 int32_t *argmax, float *max_logit, void *ws, cudaStream_t st);
+                                 int32_t *argmax, float *max_logit, void *ws, int32_t *status,
+                                 uint64_t inject_ns, cudaStream_t st);
 size_t attention_workspace_bytes(const BatchArgs &a);
 cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const uint16_t *w_qkv, int d,
                                  const float *rope_cos, const float *rope_sin, int max_pos, uint16_t *q,

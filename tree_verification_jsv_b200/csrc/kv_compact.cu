@@ -123,13 +123,11 @@ accept_compact_kernel(BatchArgs a, const int32_t *__restrict__ tokens, const int
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int32_t *row = path + (size_t)b * max_path;
 
-    // The request's geometry and page entries are read while the previous
-    // launch (the LM head) may still run: no call of this library writes
-    // prefix_len, node_offsets or page_table.  The tree, the draft tokens and
-    // the argmax (which jsv_accum_logp_tree and the LM head write), and every
-    // write to the outputs or the caches, come after the wait (the
-    // compaction overwrites cache rows that the attention reads, and the LM
-    // head completes after the attention).
+    // Every read comes after the wait for the previous launch (the LM head),
+    // the request's geometry included: a caller may pass the previous step's
+    // new_len back as prefix_len, and under programmatic dependent launch
+    // that step's compaction can still be running while this kernel starts.
+    pdl_wait_predecessor();
     Request r;
     const bool req_ok = load_request(a, b, r) && r.n <= kWalkMaxNodes;
     int par_bad = 0, bad = 0;
@@ -141,7 +139,6 @@ accept_compact_kernel(BatchArgs a, const int32_t *__restrict__ tokens, const int
             if (page < 0 || page >= a.num_pages) bad = 1;
         }
     }
-    pdl_wait_predecessor();
     if (req_ok) {
         for (int j = threadIdx.x; j < r.n; j += blockDim.x) {
             const int p = a.parent[r.base + j];
@@ -206,7 +203,7 @@ cudaError_t launch_kv_compact(const BatchArgs &a, uint16_t *k_cache, uint16_t *v
                               int32_t *new_len, cudaStream_t st) {
     dim3 grid(a.B, 2, (a.Hkv + kHeadsPerCta - 1) / kHeadsPerCta);
     size_t smem = (size_t)kCompactChunk * kHeadsPerCta * (a.D / 8) * sizeof(uint4);
-    static bool carve[64] = {};
+    static PerDeviceOnce carve;
     cudaError_t e = prefer_max_shared(kv_compact_kernel, carve);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kv_compact_kernel, grid, dim3(kCompactThreads), smem, st, a, k_cache, v_cache, path,
@@ -220,7 +217,7 @@ cudaError_t launch_accept_compact(const BatchArgs &a, const int32_t *tokens, con
                                   uint16_t *v_cache, int32_t *new_len, cudaStream_t st) {
     dim3 grid(a.B, 2, (a.Hkv + kHeadsPerCta - 1) / kHeadsPerCta);
     size_t smem = (size_t)kCompactChunk * kHeadsPerCta * (a.D / 8) * sizeof(uint4);
-    static bool carve[64] = {};
+    static PerDeviceOnce carve;
     cudaError_t e = prefer_max_shared(accept_compact_kernel, carve);
     if (e != cudaSuccess) return e;
     e = launch_pdl(accept_compact_kernel, grid, dim3(kCompactThreads), smem, st, a, tokens, argmax, max_path, path,

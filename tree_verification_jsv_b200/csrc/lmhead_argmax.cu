@@ -92,7 +92,8 @@ struct LmParams {
     unsigned int *done;        // work finished so far (zero between calls)
     int32_t *argmax;
     float *max_logit;
-    int32_t *status;
+    int32_t *status;           // device status word or NULL (JSV_ERR_TIMEOUT on a wait that gave up)
+    uint64_t inject_ns;        // failure-detection self-test: 0, or the limit of an injected wait
 };
 
 // Single-CTA form: the vocabulary is cut into `units` runs of whole 16-row
@@ -135,6 +136,24 @@ __device__ __forceinline__ void set_abort(volatile int *abort, int32_t *status) 
     if (status) atomicCAS(status, 0, JSV_ERR_TIMEOUT);
 }
 
+// The same in a CTA pair: the peer's flag is raised too (distributed shared
+// memory; both CTAs are alive until their last cluster barrier), so that both
+// stop issuing work instead of running into their own wait limits.
+__device__ __forceinline__ void set_abort_pair(volatile int *abort, int32_t *status) {
+    set_abort(abort, status);
+    st_shared_cluster_u32((const void *)abort, cluster_ctarank() ^ 1u, 1u);
+}
+
+// Failure-detection self-test (jsv_selftest_lmhead_timeout): the producer of
+// the first CTA (or CTA pair) waits, before it issues any copy, on a barrier
+// nothing signals, with the injected limit.  It gives up, reports the timeout
+// and unwinds like any timed-out wait; nothing of its own is in flight then.
+__device__ __forceinline__ bool injected_wait_gave_up(const LmParams &p, uint64_t *bar, volatile int *abort,
+                                                     unsigned first_ctas) {
+    if (p.inject_ns == 0 || blockIdx.x >= first_ctas) return false;
+    return !mbar_wait(bar, 0, abort, p.inject_ns);
+}
+
 // Answers of cluster launch control: the CTA's k-th item is blockIdx.x for
 // k = 0; the answer carrying item k + 1 lands in slot k % kClcSlots, in
 // phase (k / kClcSlots) & 1.  Every role reads every answer.
@@ -160,7 +179,7 @@ lmhead_argmax_tc_kernel(const __grid_constant__ LmWMaps tmW, const __grid_consta
     extern __shared__ uint8_t dsmem[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
     __shared__ __align__(8) uint64_t accf_bar[2], acce_bar[2], drain_bar;
-    __shared__ __align__(8) uint64_t clc_full[kClcSlots], clc_empty[kClcSlots];
+    __shared__ __align__(8) uint64_t clc_full[kClcSlots], clc_empty[kClcSlots], inject_bar;
     __shared__ __align__(16) uint4 clc_resp[kClcSlots];
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
@@ -186,6 +205,7 @@ lmhead_argmax_tc_kernel(const __grid_constant__ LmWMaps tmW, const __grid_consta
             mbar_init(&clc_empty[s], kClcReaders);
         }
         mbar_init(&drain_bar, 1);
+        mbar_init(&inject_bar, 1);
         abort_sh = 0;
         ep_fail = 0;
         claimed_sh = 1;
@@ -217,6 +237,7 @@ lmhead_argmax_tc_kernel(const __grid_constant__ LmWMaps tmW, const __grid_consta
             int item = blockIdx.x, claimed = 1;
             int pend_slot = -1;                  // an answer still on its way
             uint32_t pend_phase = 0;
+            if (injected_wait_gave_up(p, &inject_bar, &abort_sh, 1)) set_abort(&abort_sh, p.status);
             for (int k = 0; !abort_sh; ++k) {
                 const int cs = k % kClcSlots;
                 const uint32_t cph = (uint32_t)(k / kClcSlots) & 1u;
@@ -557,9 +578,11 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
     extern __shared__ uint8_t dsmem[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages], empty_bar[kMaxStages];
     __shared__ __align__(8) uint64_t accf_bar[2], acce_bar[2], drain_bar;
+    __shared__ __align__(8) uint64_t inject_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ volatile int ep_fail;
+    __shared__ int issued_sh;                         // K-chunk stages this CTA's producer issued
     __shared__ unsigned long long red[kEpiWarps][kMaxGroupNodes];
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
@@ -579,8 +602,10 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
             mbar_init(&acce_bar[a], 2 * kEpiWarps);   // epilogue warps of both CTAs
         }
         mbar_init(&drain_bar, 1);
+        mbar_init(&inject_bar, 1);
         abort_sh = 0;
         ep_fail = 0;
+        issued_sh = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -604,7 +629,8 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
             const uint64_t pol_h = policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
-            long long issued = 0;
+            int issued = 0;
+            if (injected_wait_gave_up(p, &inject_bar, &abort_sh, 2)) set_abort_pair(&abort_sh, p.status);
             for (int it = 0; it < items && !abort_sh; ++it) {
                 const LmPairItem t = work.item(p, it);
                 const int my_rows = pair_rows(t, rank);
@@ -617,7 +643,7 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
                 bool ok = true;
                 for (int kc = 0; kc < p.kchunks; ++kc) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh)) {
-                        set_abort(&abort_sh, p.status);
+                        set_abort_pair(&abort_sh, p.status);
                         ok = false;
                         break;
                     }
@@ -638,18 +664,7 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
                 }
                 if (!ok) break;
             }
-            if (abort_sh && rank == 0) {
-                // let every load still in flight (both CTAs') land before exit
-                int zero = 0;
-                const long long back = issued < p.stages ? issued : p.stages;
-                int s = stage;
-                uint32_t ph = phase;
-                for (long long i = 0; i < back; ++i) {
-                    if (s == 0) { s = p.stages; ph ^= 1; }
-                    --s;
-                    mbar_wait(&full_bar[s], ph, (volatile int *)&zero);
-                }
-            }
+            issued_sh = issued;
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
@@ -669,7 +684,7 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
                 const int acc = it & 1;
                 const uint32_t use = (uint32_t)(it >> 1);
                 if (!wait1(&acce_bar[acc], (use & 1) ^ 1)) {
-                    if (lane == 0) set_abort(&abort_sh, p.status);
+                    if (lane == 0) set_abort_pair(&abort_sh, p.status);
                     break;
                 }
                 tc_fence_after();
@@ -679,7 +694,7 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
                 bool ok = true;
                 for (int kc = 0; kc < p.kchunks; ++kc) {
                     if (!wait1(&full_bar[stage], phase)) {
-                        if (lane == 0) set_abort(&abort_sh, p.status);
+                        if (lane == 0) set_abort_pair(&abort_sh, p.status);
                         ok = false;
                         break;
                     }
@@ -713,7 +728,7 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
             const int acc = it & 1;
             const uint32_t use = (uint32_t)(it >> 1);
             if (!mbar_wait(&accf_bar[acc], use & 1, &abort_sh)) {
-                set_abort(&abort_sh, p.status);
+                set_abort_pair(&abort_sh, p.status);
                 ep_fail = 1;
             }
             named_barrier(1, 32 * kEpiWarps);
@@ -769,7 +784,33 @@ lmhead_argmax_pair_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_
     __syncwarp();
     tc_fence_before();
     __threadfence();
-    cluster_sync();          // both CTAs done with the pair's TMEM and shared memory
+    cluster_sync();          // both CTAs done with the pair's TMEM; producers' issue counts published
+    // After an abort, copies may still be in flight into either CTA's shared
+    // memory.  Every copy of a stage completes on the first CTA's barrier, so
+    // its producer waits for each stage either CTA issued (the last `stages`
+    // of them), first completing by hand the bytes of a CTA that never issued
+    // its part of that stage and arming a stage only the second CTA issued.
+    // Both CTAs then meet again, so neither exits with its copies in flight.
+    const bool any_abort = abort_sh || ld_shared_cluster_u32((const void *)&abort_sh, (uint32_t)rank ^ 1u);
+    if (any_abort) {
+        if (rank == 0 && warp == 0 && lane == 0) {
+            const int n0 = issued_sh, n1 = (int)ld_shared_cluster_u32(&issued_sh, 1);
+            const int n = n0 > n1 ? n0 : n1;
+            int zero = 0;
+            for (int i = n - p.stages > 0 ? n - p.stages : 0; i < n; ++i) {
+                const int s = i % p.stages;
+                const uint32_t ph = (uint32_t)((i / p.stages) & 1);
+                const LmPairItem t = work.item(p, i / p.kchunks);
+                const uint32_t b0 = (uint32_t)half_nodes * 128 + w_bytes(pair_rows(t, 0));
+                const uint32_t b1 = (uint32_t)half_nodes * 128 + (pair_rows(t, 1) > 0 ? w_bytes(pair_rows(t, 1)) : 0u);
+                if (i >= n0) mbar_arrive_expect_tx(&full_bar[s], b1);      // armed by neither: rank 1's part only
+                else if (i >= n1) mbar_complete_tx(&full_bar[s], b1);      // rank 1's part never issued
+                mbar_wait(&full_bar[s], ph, (volatile int *)&zero);
+            }
+        }
+        __syncwarp();
+        cluster_sync();
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem, 512);
@@ -798,10 +839,14 @@ size_t lmhead_workspace_bytes(int T, int d, int V) {
 // Pairs of CTAs that can be resident at once for a given dynamic shared memory
 // size (0 if clusters cannot be used).
 static int pair_clusters(size_t smem) {
-    static int cache[64] = {0};
+    // several host threads may fill an entry at once; they store the same value
+    static std::atomic<int> cache[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
-    if (dev < 64 && cache[dev]) return cache[dev];
+    if (dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c) return c > 0 ? c : 0;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 256);
     cfg.blockDim = dim3(kLmThreads);
@@ -818,13 +863,13 @@ static int pair_clusters(size_t smem) {
         cudaGetLastError();
         n = 0;
     }
-    if (dev < 64) cache[dev] = n > 0 ? n : -1;
+    if (dev < 64) cache[dev].store(n > 0 ? n : -1, std::memory_order_relaxed);
     return n > 0 ? n : 0;
 }
 
 cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int T, int d, int V,
-                                 int32_t *argmax, float *max_logit, void *ws, cudaStream_t st) {
-    int32_t *status = nullptr;
+                                 int32_t *argmax, float *max_logit, void *ws, int32_t *status,
+                                 uint64_t inject_ns, cudaStream_t st) {
     auto *keys = static_cast<unsigned long long *>(ws);
     LmParams p;
     p.T = T; p.d = d; p.V = V;
@@ -836,11 +881,10 @@ cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int 
     p.argmax = argmax;
     p.max_logit = max_logit;
     p.status = status;
+    p.inject_ns = inject_ns;
 
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    static PerDeviceOnce attr_once;
+    cudaError_t ae = attr_once.run([]() {
         cudaError_t e = cudaFuncSetAttribute(lmhead_argmax_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kSmemBudget + 1024);
         if (e == cudaSuccess)
@@ -852,9 +896,9 @@ cudaError_t launch_lmhead_argmax(const uint16_t *hidden, const uint16_t *w, int 
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(lmhead_argmax_pair_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                      (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+        return e;
+    });
+    if (ae != cudaSuccess) return ae;
     int sms = device_sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
 

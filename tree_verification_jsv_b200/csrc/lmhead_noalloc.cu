@@ -26,9 +26,10 @@ static __device__ __align__(256) unsigned long long g_lmhead_noalloc_keys[JSV_NO
 namespace {
 std::mutex g_noalloc_mu;
 void *g_noalloc_addr[64] = {nullptr};
+}  // namespace
 
-// Device address of the scratch array on the current device (set-up on
-// the first call made with that device current).
+// Device address of the scratch array on the current device (set-up on the
+// first call made with that device current).
 cudaError_t noalloc_scratch(void **out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -44,27 +45,26 @@ cudaError_t noalloc_scratch(void **out) {
     *out = g_noalloc_addr[dev];
     return cudaSuccess;
 }
-}  // namespace
 
 }  // namespace jsv
 
 extern "C" {
 
 jsv_status jsv_lmhead_argmax_noalloc(const uint16_t *hidden, const uint16_t *w, int32_t T, int32_t d,
-                                     int32_t V, int32_t *argmax, float *max_logit, void *stream) {
-    if (!hidden || !w || !argmax || T < 1 || d < 1 || V < 1) return JSV_ERR_INVALID_ARG;
+                                     int32_t V, int32_t *argmax, float *max_logit, int32_t *dev_status,
+                                     void *stream) {
+    jsv_status s = jsv::check_lmhead_args(hidden, w, T, d, V, argmax);
+    if (s != JSV_OK) return s;
     if (T > JSV_NOALLOC_MAX_NODES) return JSV_ERR_UNSUPPORTED;
-    if (d % 64 != 0 || d > 16384) return JSV_ERR_UNSUPPORTED;
-    if ((reinterpret_cast<uintptr_t>(hidden) % 16) || (reinterpret_cast<uintptr_t>(w) % 16))
-        return JSV_ERR_INVALID_ARG;
     void *scratch = nullptr;
-    if (jsv::noalloc_scratch(&scratch) != cudaSuccess) return JSV_ERR_CUDA;
-    // the array is zero at load and every call leaves its keys and counter zeroed
+    s = jsv::from_cuda(jsv::noalloc_scratch(&scratch));
+    if (s != JSV_OK) return s;
+    // the array is zero at load and every call leaves its keys and counter
+    // zeroed, a call that timed out included
     static_assert(sizeof(jsv::g_lmhead_noalloc_keys) >= (JSV_NOALLOC_MAX_NODES + 1) * sizeof(unsigned long long),
                   "scratch must hold the keys and the completion counter");
-    cudaError_t e = jsv::launch_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, scratch,
-                                              static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? JSV_OK : JSV_ERR_CUDA;
+    return jsv::from_cuda(jsv::launch_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, scratch, dev_status, 0,
+                                                    static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -364,18 +364,16 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
     if (!encode_tensor_map_2d(&tmX, x, (uint64_t)d, (uint64_t)a.total_nodes, (uint64_t)d * 2, kQKChunk, p.box_rows))
         return cudaErrorInvalidValue;
     const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    static PerDeviceOnce attr_once;
+    cudaError_t ae = attr_once.run([]() {
         cudaError_t e = cudaFuncSetAttribute(qkv_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kQSmemBudget + 1024);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(qkv_rope_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                      (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+        return e;
+    });
+    if (ae != cudaSuccess) return ae;
     const int tiles = (p.rows_total + kQTileM - 1) / kQTileM;
     const int groups = (a.total_nodes + p.group_nodes - 1) / p.group_nodes;
     // Too few (tile, group) CTAs to stream the weight with every SM: split K

@@ -1,4 +1,4 @@
-// Failure-detection self-test for the bounded device waits.
+// Failure-detection self-tests for the bounded device waits.
 //
 // Every wait of the library's tcgen05 kernels on an mbarrier gives up after
 // a wall-clock limit, sets an error code and unwinds, so a lost arrival
@@ -34,4 +34,28 @@ extern "C" jsv_status jsv_selftest_wait_timeout(int32_t *dev_status, uint32_t li
         dev_status, (uint64_t)limit_us * 1000ull);
     jsv::count_launches(1);
     return cudaGetLastError() == cudaSuccess ? JSV_OK : JSV_ERR_CUDA;
+}
+
+// The LM head with one injected wait that gives up (see jsv.h): the same
+// launch as jsv_lmhead_argmax (workspace given) or jsv_lmhead_argmax_noalloc
+// (workspace NULL), with the first CTA's producer stalled on a barrier that
+// nothing signals before it issues any copy.
+extern "C" jsv_status jsv_selftest_lmhead_timeout(const uint16_t *hidden, const uint16_t *w, int32_t T, int32_t d,
+                                                  int32_t V, int32_t *argmax, float *max_logit, void *workspace,
+                                                  size_t workspace_bytes, int32_t *dev_status, uint32_t limit_us,
+                                                  void *stream) {
+    jsv_status s = jsv::check_lmhead_args(hidden, w, T, d, V, argmax);
+    if (s != JSV_OK) return s;
+    if (!dev_status || limit_us < 1 || limit_us > 2000000) return JSV_ERR_INVALID_ARG;
+    if (workspace) {
+        if (workspace_bytes < jsv::lmhead_workspace_bytes(T, d, V) ||
+            (reinterpret_cast<uintptr_t>(workspace) % 8) != 0)
+            return JSV_ERR_INVALID_ARG;
+    } else {
+        if (T > JSV_NOALLOC_MAX_NODES) return JSV_ERR_UNSUPPORTED;
+        s = jsv::from_cuda(jsv::noalloc_scratch(&workspace));
+        if (s != JSV_OK) return s;
+    }
+    return jsv::from_cuda(jsv::launch_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, workspace, dev_status,
+                                                    (uint64_t)limit_us * 1000ull, static_cast<cudaStream_t>(stream)));
 }

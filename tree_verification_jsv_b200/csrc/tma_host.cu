@@ -5,6 +5,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 namespace jsv {
@@ -52,13 +53,17 @@ bool encode_tensor_map_3d(CUtensorMap *map, const void *base, uint64_t d0, uint6
 }
 
 int device_sm_count() {
-    static int cache[64] = {0};
+    // several host threads may fill an entry at once; they store the same value
+    static std::atomic<int> cache[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
-    if (dev < 64 && cache[dev]) return cache[dev];
+    if (dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c) return c;
+    }
     int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (dev < 64) cache[dev] = n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 0;
+    if (dev < 64 && n > 0) cache[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 

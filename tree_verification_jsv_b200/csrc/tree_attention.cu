@@ -850,18 +850,16 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
     if (!encode_tensor_map_3d(&tmV, v_cache, D, a.Hkv, slots, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2, 64, 1, 16))
         return cudaErrorInvalidValue;
     const size_t smem = (size_t)Lt::kTotal + 1024;
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    static PerDeviceOnce attr_once;
+    cudaError_t ae = attr_once.run([&]() {
         cudaError_t e = cudaFuncSetAttribute(tree_attention_tc_kernel<D>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(tree_attention_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                      (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+        return e;
+    });
+    if (ae != cudaSuccess) return ae;
     dim3 grid((a.max_nodes * G + kRowsPerCta - 1) / kRowsPerCta, S, a.B * a.Hkv);
     cudaError_t le = launch_pdl(tree_attention_tc_kernel<D>, grid, dim3(kAttnThreads), smem, st, tmK, tmV, tmQ, prm);
     if (le != cudaSuccess) {
@@ -872,7 +870,7 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
         return le;
     }
     dim3 cgrid((a.max_nodes * G + kCombineWarps - 1) / kCombineWarps, 1, a.B * a.Hkv);
-    static bool carve[64] = {};
+    static PerDeviceOnce carve;
     le = prefer_max_shared(tree_attention_combine_kernel<D>, carve);
     if (le != cudaSuccess) return le;
     le = launch_pdl(tree_attention_combine_kernel<D>, cgrid, dim3(kCombineWarps * 32), 0, st, a, S,

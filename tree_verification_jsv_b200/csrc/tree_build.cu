@@ -271,18 +271,16 @@ cudaError_t launch_accum_logp_tree(const float *logp, const int32_t *topk_tokens
                                    float *score, int32_t *num_nodes, int32_t *status, cudaStream_t st) {
     TreeArgs a{logp, topk_tokens, root_token, B, D, k, budget, parent, tokens, depth, score, num_nodes, status};
     const size_t smem = (size_t)kTreeWarps * 2 * kTreeLevel * sizeof(float);
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    static PerDeviceOnce attr_once;
+    cudaError_t ae = attr_once.run([&]() {
         cudaError_t e = cudaFuncSetAttribute(accum_logp_tree_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(accum_logp_tree_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                      (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+        return e;
+    });
+    if (ae != cudaSuccess) return ae;
     cudaError_t e = launch_pdl(accum_logp_tree_kernel, dim3(B), dim3(32 * kTreeWarps), smem, st, a);
     count_launches(1);
     return e;

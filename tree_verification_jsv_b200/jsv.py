@@ -24,6 +24,7 @@ EXPORTS = ("jsv_tree_attention_workspace_size", "jsv_tree_attention",
            "jsv_lmhead_argmax_workspace_size", "jsv_lmhead_argmax", "jsv_accept_path",
            "jsv_kv_compact", "jsv_status_string", "jsv_version", "jsv_kernel_launches",
            "jsv_lmhead_argmax_noalloc", "jsv_last_error_string", "jsv_selftest_wait_timeout",
+           "jsv_selftest_lmhead_timeout",
            "jsv_accum_logp_tree", "jsv_tree_qkv_rope", "jsv_accept_compact")
 
 # Largest node count jsv_lmhead_argmax_noalloc accepts (JSV_NOALLOC_MAX_NODES).
@@ -70,7 +71,7 @@ def load() -> ctypes.CDLL:
     lib.jsv_tree_attention.restype = ctypes.c_int
     lib.jsv_lmhead_argmax_workspace_size.argtypes = [i32, i32, i32]
     lib.jsv_lmhead_argmax_workspace_size.restype = sz
-    lib.jsv_lmhead_argmax.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]
+    lib.jsv_lmhead_argmax.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp, vp]
     lib.jsv_lmhead_argmax.restype = ctypes.c_int
     lib.jsv_accept_path.argtypes = [bp, vp, vp, i32, vp, vp, vp, vp]
     lib.jsv_accept_path.restype = ctypes.c_int
@@ -82,7 +83,7 @@ def load() -> ctypes.CDLL:
     lib.jsv_status_string.restype = ctypes.c_char_p
     lib.jsv_version.argtypes = []
     lib.jsv_version.restype = i32
-    lib.jsv_lmhead_argmax_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp]
+    lib.jsv_lmhead_argmax_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp]
     lib.jsv_lmhead_argmax_noalloc.restype = ctypes.c_int
     lib.jsv_tree_qkv_rope.argtypes = [bp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp]
     lib.jsv_tree_qkv_rope.restype = ctypes.c_int
@@ -90,6 +91,8 @@ def load() -> ctypes.CDLL:
     lib.jsv_accum_logp_tree.restype = ctypes.c_int
     lib.jsv_selftest_wait_timeout.argtypes = [vp, ctypes.c_uint32, vp]
     lib.jsv_selftest_wait_timeout.restype = ctypes.c_int
+    lib.jsv_selftest_lmhead_timeout.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, sz, vp, ctypes.c_uint32, vp]
+    lib.jsv_selftest_lmhead_timeout.restype = ctypes.c_int
     lib.jsv_last_error_string.argtypes = []
     lib.jsv_last_error_string.restype = ctypes.c_char_p
     lib.jsv_kernel_launches.argtypes = []
@@ -159,22 +162,36 @@ def jsv_lmhead_argmax_workspace_size(T, d, V) -> int:
     return int(load().jsv_lmhead_argmax_workspace_size(int(T), int(d), int(V)))
 
 
+def _nbytes(buf, nbytes):
+    if nbytes is not None:
+        return int(nbytes)
+    return 0 if buf is None or isinstance(buf, int) else buf.numel() * buf.element_size()
+
+
 def jsv_lmhead_argmax(hidden, w, T, d, V, argmax, max_logit, workspace, workspace_bytes=None,
-                      stream=None) -> None:
-    if workspace_bytes is None:
-        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+                      dev_status=None, stream=None) -> None:
     st = load().jsv_lmhead_argmax(_addr(hidden), _addr(w), int(T), int(d), int(V), _addr(argmax),
-                                  _addr(max_logit), _addr(workspace), int(workspace_bytes),
-                                  _stream(stream))
+                                  _addr(max_logit), _addr(workspace), _nbytes(workspace, workspace_bytes),
+                                  _addr(dev_status), _stream(stream))
     _check("jsv_lmhead_argmax", st)
 
 
-def jsv_lmhead_argmax_noalloc(hidden, w, T, d, V, argmax, max_logit, stream=None) -> None:
+def jsv_lmhead_argmax_noalloc(hidden, w, T, d, V, argmax, max_logit, dev_status=None, stream=None) -> None:
     """LM-head argmax with the library's fixed scratch (no workspace, no
     allocation); see include/jsv.h for its limits and sharing rules."""
     st = load().jsv_lmhead_argmax_noalloc(_addr(hidden), _addr(w), int(T), int(d), int(V),
-                                          _addr(argmax), _addr(max_logit), _stream(stream))
+                                          _addr(argmax), _addr(max_logit), _addr(dev_status), _stream(stream))
     _check("jsv_lmhead_argmax_noalloc", st)
+
+
+def jsv_selftest_lmhead_timeout(hidden, w, T, d, V, argmax, max_logit, workspace, dev_status, limit_us,
+                                workspace_bytes=None, stream=None) -> None:
+    """The LM head with one injected wait that gives up (see include/jsv.h);
+    ``workspace=None`` runs it on the no-alloc entry point's scratch array."""
+    st = load().jsv_selftest_lmhead_timeout(_addr(hidden), _addr(w), int(T), int(d), int(V), _addr(argmax),
+                                            _addr(max_logit), _addr(workspace), _nbytes(workspace, workspace_bytes),
+                                            _addr(dev_status), int(limit_us), _stream(stream))
+    _check("jsv_selftest_lmhead_timeout", st)
 
 
 def jsv_tree_qkv_rope(batch, x, w_qkv, d, rope_cos, rope_sin, max_pos, q, k_cache, v_cache,

@@ -106,7 +106,7 @@ class VerifyStep:
             node_offsets=self.node_offsets, parent=self.parent, dev_status=self.status)
         aws = jsv.jsv_tree_attention_workspace_size(self.batch)
         lws = jsv.jsv_lmhead_argmax_workspace_size(self.T, self.d, self.V)
-        self.attn_ws = torch.empty(max(aws, 256), dtype=torch.uint8, device=dev)
+        self.attn_ws = torch.zeros(max(aws, 256), dtype=torch.uint8, device=dev)   # zeroed once; each call leaves it ready
         self.lm_ws = torch.zeros(max(lws, 8), dtype=torch.uint8, device=dev)   # zeroed once; each call leaves it zeroed
         self._graph = None
 
@@ -117,7 +117,7 @@ class VerifyStep:
 
     def lmhead(self, stream=None):
         jsv.jsv_lmhead_argmax(self.hidden, self.w, self.T, self.d, self.V, self.argmax,
-                              self.max_logit, self.lm_ws, stream=stream)
+                              self.max_logit, self.lm_ws, dev_status=self.status, stream=stream)
 
     def accept(self, stream=None):
         jsv.jsv_accept_path(self.batch, self.tokens, self.argmax, self.max_path, self.path,
