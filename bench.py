@@ -540,9 +540,23 @@ def run_gpu(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize()
         assert int(st.status.item()) == 0
+        eager_us = 1e3 * e0.elapsed_time(e1) / args.steps
+        # the same calls from one CUDA graph: device time without host launch gaps
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(args.steps):
+                call()
+        graph.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        assert int(st.status.item()) == 0
         gb.clocks.stop()
-        print(json.dumps({"profile": args.profile, "workload": args.workload,
-                          "mean_us_warm_l2": 1e3 * e0.elapsed_time(e1) / args.steps}), flush=True)
+        print(json.dumps({"profile": args.profile, "workload": args.workload, "mean_us_warm_l2": eager_us,
+                          "graph_us_warm_l2": 1e3 * e0.elapsed_time(e1) / args.steps}), flush=True)
+        del graph
         return
 
     # correctness of this very launch configuration against stored oracle values

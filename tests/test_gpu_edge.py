@@ -77,6 +77,15 @@ ATTN_CASES = {
     "g5_two_row_tiles": ([synth.budget_tree(np.random.default_rng(6), 60, 8, 4)], [700], 10, 2, 128),
     "g3_head_dim_64": ([synth.tiny_tree(np.random.default_rng(7), 50, 6, 3),
                         synth.tiny_tree(np.random.default_rng(8), 9, 3, 2)], [130, 33], 6, 2, 64),
+    # a ragged batch: the two long requests take several KV splits (merged by
+    # the combine kernel) while the short ones take one split each and are
+    # written straight from the attention kernel
+    "short_and_long_mix": ([np.arange(-1, 30)] + [synth.tiny_tree(np.random.default_rng(20 + i), 5 + i, 4, 3)
+                                                  for i in range(18)] + [np.arange(-1, 9)],
+                           [8000] + [50 + 7 * i for i in range(18)] + [5003], 8, 2, 128),
+    # G = 16 (Q by TMA, 8 nodes per 128-row group), a prefix ending inside a
+    # page and a 256-node tree whose tiles fall into more than one split
+    "g16_tree_cut": ([synth.budget_tree(np.random.default_rng(9), 256, 16, 8)], [2077], 16, 1, 128),
 }
 
 
@@ -90,6 +99,35 @@ def test_attention_edge_cases(name, sharp):
     assert st == 0
     from helpers import run_oracle_attention
     attention_close(got, run_oracle_attention(case), name)
+
+
+def test_attention_workspace_reused_without_clearing():
+    """One attention workspace, filled with garbage once, serves calls of
+    different batch shapes back to back on one stream: no call may depend on
+    what an earlier call (of another geometry and split count) left in it."""
+    names = ["short_and_long_mix", "g8_long", "short_and_long_mix", "g16_tree_cut", "chain_cross_pages"]
+    cases, outs, sizes = [], [], []
+    for i, name in enumerate(names):
+        parents, pre, Hq, Hkv, D = ATTN_CASES[name]
+        cases.append(small_case(parents, pre, Hq=Hq, Hkv=Hkv, D=D, seed=40 + i))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    batches = [_batch(c, status) for c in cases]
+    sizes = [jsv.jsv_tree_attention_workspace_size(b) for b, _ in batches]
+    ws = torch.full((max(max(sizes), 256),), 0x5A, dtype=torch.uint8, device="cuda")
+    keep = []
+    for c, (b, dev) in zip(cases, batches):
+        q, k, v = _dev_bf16(c["q"]), _dev_bf16(c["k_cache"]), _dev_bf16(c["v_cache"])
+        T = int(c["node_offsets"][-1])
+        out = torch.zeros((T, c["Hq"], c["D"]), dtype=torch.bfloat16, device="cuda")
+        jsv.jsv_tree_attention(b, q, k, v, c["scale"], out, ws)
+        keep.append((q, k, v, dev))
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    from helpers import run_oracle_attention
+    for name, c, out in zip(names, cases, outs):
+        got = synth.bf16_bits_to_f32(_bits(out)).astype(np.float64)
+        attention_close(got, run_oracle_attention(c), name)
 
 
 # (64, 128, 40000): single CTAs with vocabulary units of 8 or 9 boxes, i.e.

@@ -107,12 +107,20 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 struct AttnParams {
     BatchArgs a;
     const uint16_t *q;
+    uint16_t *out;         // [T][Hq][D] bf16, written here for rows that are not split
     float scale_log2;
-    int S;                 // splits
+    int S;                 // most splits of a request (grid dimension y)
+    int C;                 // key tiles a split aims at
     int q_tma;             // 1: Q is copied by TMA (G divides 128), 0: by the softmax warps
     float *ws_o;           // [S][T*Hq][D]
     float *ws_ml;          // [S][T*Hq][2]
 };
+
+// Splits of a request with `total` key tiles: about C tiles each, at most S,
+// so that short requests of a ragged batch take fewer CTAs than long ones.
+__device__ __forceinline__ int request_splits(int total, int C, int S) {
+    return max(1, min(S, (total + C - 1) / C));
+}
 
 template <int D>
 struct AttnSmem {
@@ -250,6 +258,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     __shared__ __align__(8) uint64_t s_full[kGroups], p_full[kGroups], o_done[kGroups], q_ready, drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
+    __shared__ int direct_sh;              // 1: the request has one split (rows written here in bf16)
     __shared__ uint32_t anc[kRowsPerCta][kMaxTreeWords];
     __shared__ int par_sh[32 * kMaxTreeWords];
 
@@ -268,13 +277,15 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     const int ngroups = rows_here > kGroupRows ? 2 : 1;     // a group with no rows is skipped
 
     // tile schedule for this split
-    // Logical tiles: the prefix tiles, then the tree tiles; split s takes the
-    // balanced run [total * s / S, total * (s + 1) / S).
+    // Logical tiles: the prefix tiles, then the tree tiles; of the request's
+    // Sb splits, split s takes the balanced run [total * s / Sb, total * (s + 1) / Sb).
     const int prefix_tiles = (r.P + kKeyTile - 1) / kKeyTile;
     const int P0 = r.P & ~15;                    // tree tiles start on a page boundary
     const int total_tiles = prefix_tiles + (r.P + r.n - P0 + kKeyTile - 1) / kKeyTile;
-    const int t_begin = (int)((long long)total_tiles * split / prm.S);
-    const int t_end = (int)((long long)total_tiles * (split + 1) / prm.S);
+    const int Sb = request_splits(total_tiles, prm.C, prm.S);
+    if (split >= Sb) return;
+    const int t_begin = (int)((long long)total_tiles * split / Sb);
+    const int t_end = (int)((long long)total_tiles * (split + 1) / Sb);
     const int ntiles = t_end - t_begin;
     const int tree_tiles = max(0, t_end - max(t_begin, prefix_tiles));    // tree tiles of this split
 
@@ -299,6 +310,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         mbar_init(&q_ready, 4 * kGroups + 1);     // softmax warps + the producer
         mbar_init(&drain_bar, 1);
         abort_sh = 0;
+        direct_sh = Sb == 1 ? 1 : 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -669,16 +681,21 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         }
         const size_t rows = (size_t)a.total_nodes * a.Hq;
         const size_t row_id = (size_t)(r.base + min(node, r.n - 1)) * a.Hq + head;
-        // The partial is written through shared memory so that global stores are
-        // whole rows: each warp stages its 32 rows, half of D at a time, in its
-        // own slice of this group's Q buffer (free once the group's last product
+        // A request with one split writes its rows here, normalised, in bf16;
+        // otherwise this split's partial goes to the workspace in fp32.  Either
+        // is written through shared memory so that global stores are whole
+        // rows: each warp stages its 32 rows, half of D at a time, in its own
+        // slice of this group's Q buffer (free once the group's last product
         // has completed: every product of the group precedes its last PV), XOR-
         // swizzled by row so that neither side of the transpose has bank conflicts.
+        const bool direct = direct_sh != 0;
+        const float row_scale = direct ? (l > 0.f ? 1.f / l : 0.f) : 1.f;
         constexpr int kScrCols = D / 2;
         constexpr int kChunks = kScrCols / 4;                   // 16-byte chunks per staged row
         constexpr int kRowsPerStore = 32 / kChunks;
         float4 *scr = reinterpret_cast<float4 *>(sQ + grp * L::kQGroupBytes + sub * (32 * kScrCols * 4));
-        const long long my_off = row_valid ? (long long)(((size_t)split * rows + row_id) * D) : -1ll;
+        const long long my_off =
+            row_valid ? (long long)((direct ? row_id : (size_t)split * rows + row_id) * D) : -1ll;
         if (have_o) tc_fence_after();
 #pragma unroll
         for (int pass = 0; pass < 2; ++pass) {
@@ -695,8 +712,9 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 #pragma unroll
                 for (int x = 0; x < 8; ++x)
                     scr[lane * kChunks + ((c0 / 4 + x) ^ (lane & (kChunks - 1)))] =
-                        make_float4(__uint_as_float(rr[4 * x]), __uint_as_float(rr[4 * x + 1]),
-                                    __uint_as_float(rr[4 * x + 2]), __uint_as_float(rr[4 * x + 3]));
+                        make_float4(__uint_as_float(rr[4 * x]) * row_scale, __uint_as_float(rr[4 * x + 1]) * row_scale,
+                                    __uint_as_float(rr[4 * x + 2]) * row_scale,
+                                    __uint_as_float(rr[4 * x + 3]) * row_scale);
             }
             __syncwarp();
 #pragma unroll 4
@@ -704,11 +722,16 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 const int wr = i + lane / kChunks, ch = lane % kChunks;
                 const long long off = __shfl_sync(0xffffffffu, my_off, wr);
                 const float4 v = scr[wr * kChunks + (ch ^ (wr & (kChunks - 1)))];
-                if (off >= 0) *reinterpret_cast<float4 *>(prm.ws_o + off + pass * kScrCols + ch * 4) = v;
+                if (off < 0) continue;
+                if (direct)
+                    *reinterpret_cast<uint2 *>(prm.out + off + pass * kScrCols + ch * 4) =
+                        make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+                else
+                    *reinterpret_cast<float4 *>(prm.ws_o + off + pass * kScrCols + ch * 4) = v;
             }
             __syncwarp();
         }
-        if (row_valid) {
+        if (row_valid && !direct) {
             prm.ws_ml[((size_t)split * rows + row_id) * 2 + 0] = m_used;
             prm.ws_ml[((size_t)split * rows + row_id) * 2 + 1] = l;
         }
@@ -732,7 +755,7 @@ constexpr int kCombineWarps = 4;
 
 template <int D>
 __global__ void __launch_bounds__(kCombineWarps * 32, 16)
-tree_attention_combine_kernel(BatchArgs a, int S, const float *__restrict__ ws_o,
+tree_attention_combine_kernel(BatchArgs a, int S_max, int C, const float *__restrict__ ws_o,
                               const float *__restrict__ ws_ml, uint16_t *__restrict__ out) {
     pdl_allow_dependents();
     pdl_wait_predecessor();
@@ -744,6 +767,9 @@ tree_attention_combine_kernel(BatchArgs a, int S, const float *__restrict__ ws_o
     Request r;
     if (!load_request(a, b, r)) return;
     if (rloc >= r.n * G) return;
+    const int total_tiles = (r.P + kKeyTile - 1) / kKeyTile + (r.P + r.n - (r.P & ~15) + kKeyTile - 1) / kKeyTile;
+    const int S = request_splits(total_tiles, C, S_max);
+    if (S == 1) return;                              // the attention kernel wrote these rows
     const int i = rloc / G, h = g * G + rloc % G, t = r.base + i;
     const size_t row_id = (size_t)t * a.Hq + h;
     const size_t rows = (size_t)a.total_nodes * a.Hq;
@@ -793,17 +819,24 @@ tree_attention_combine_kernel(BatchArgs a, int S, const float *__restrict__ ws_o
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+// Key tiles of the largest request the batch may hold (a bound on every
+// request's prefix + tree tiles).
+static int max_request_tiles(const BatchArgs &a) {
+    return (a.max_prefix + kKeyTile - 1) / kKeyTile + (a.max_nodes + 15 + kKeyTile - 1) / kKeyTile;
+}
+
 static int attention_splits(const BatchArgs &a) {
-    // Choose S to minimise an estimate of the kernel time in tile periods
-    // (about 2.3 us each): waves(S) * (kFixed + ceil(total / S)) plus, per
-    // split, the write and read of its fp32 partial at about 6 TB/s, where
-    // total = prefix tiles + tree tiles of the largest request, a wave is one
-    // CTA per SM and kFixed covers set-up, the first loads and the partial
-    // write of a CTA.
+    // Choose S, the splits of the largest request, to minimise an estimate of
+    // the kernel time in tile periods (about 2.3 us each): waves(S) * (kFixed
+    // + ceil(total / S)) plus, per split, the write and read of its fp32
+    // partial at about 6 TB/s, where total = prefix tiles + tree tiles of the
+    // largest request, a wave is one CTA per SM and kFixed covers set-up, the
+    // first loads and the partial write of a CTA.  (Shorter requests take
+    // proportionally fewer splits, so the estimate is an upper bound.)
     const int G = a.Hq / a.Hkv;
     const int mtiles = (a.max_nodes * G + kRowsPerCta - 1) / kRowsPerCta;
     const long long units = (long long)a.B * a.Hkv * mtiles;
-    const int total = (a.max_prefix + kKeyTile - 1) / kKeyTile + (a.max_nodes + 15 + kKeyTile - 1) / kKeyTile;
+    const int total = max_request_tiles(a);
     const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
     const double kFixed = 3.0, kTileUs = 2.3;
     const double comb = (double)a.total_nodes * a.Hq * (a.D + 2) * 4.0 * 2.0 / 6.0e6 / kTileUs;   // per split
@@ -819,7 +852,8 @@ static int attention_splits(const BatchArgs &a) {
 
 size_t attention_workspace_bytes(const BatchArgs &a) {
     const size_t rows = (size_t)a.total_nodes * a.Hq;
-    return (size_t)attention_splits(a) * rows * ((size_t)a.D + 2) * sizeof(float);
+    const int S = attention_splits(a);
+    return S > 1 ? (size_t)S * rows * ((size_t)a.D + 2) * sizeof(float) : 0;   // one split: no partials
 }
 
 template <int D>
@@ -832,10 +866,12 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
     AttnParams prm;
     prm.a = a;
     prm.q = q;
+    prm.out = out;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.S = S;
-    prm.ws_o = static_cast<float *>(ws);
-    prm.ws_ml = prm.ws_o + (size_t)S * rows * D;
+    prm.C = (max_request_tiles(a) + S - 1) / S;
+    prm.ws_o = S > 1 ? static_cast<float *>(ws) : nullptr;
+    prm.ws_ml = S > 1 ? prm.ws_o + (size_t)S * rows * D : nullptr;
 
     CUtensorMap tmK, tmV, tmQ;
     memset(&tmQ, 0, sizeof(tmQ));
@@ -869,11 +905,15 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
                                 fa.maxDynamicSharedSizeBytes, kAttnThreads, smem);
         return le;
     }
+    if (S == 1) {                 // every row was written by the attention kernel
+        count_launches(1);
+        return cudaSuccess;
+    }
     dim3 cgrid((a.max_nodes * G + kCombineWarps - 1) / kCombineWarps, 1, a.B * a.Hkv);
     static PerDeviceOnce carve;
     le = prefer_max_shared(tree_attention_combine_kernel<D>, carve);
     if (le != cudaSuccess) return le;
-    le = launch_pdl(tree_attention_combine_kernel<D>, cgrid, dim3(kCombineWarps * 32), 0, st, a, S,
+    le = launch_pdl(tree_attention_combine_kernel<D>, cgrid, dim3(kCombineWarps * 32), 0, st, a, S, prm.C,
                     (const float *)prm.ws_o, (const float *)prm.ws_ml, out);
     count_launches(2);
     return le;

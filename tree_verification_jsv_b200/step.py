@@ -106,7 +106,7 @@ class VerifyStep:
             node_offsets=self.node_offsets, parent=self.parent, dev_status=self.status)
         aws = jsv.jsv_tree_attention_workspace_size(self.batch)
         lws = jsv.jsv_lmhead_argmax_workspace_size(self.T, self.d, self.V)
-        self.attn_ws = torch.zeros(max(aws, 256), dtype=torch.uint8, device=dev)   # zeroed once; each call leaves it ready
+        self.attn_ws = torch.zeros(max(aws, 256), dtype=torch.uint8, device=dev)   # any contents: every call writes what it reads
         self.lm_ws = torch.zeros(max(lws, 8), dtype=torch.uint8, device=dev)   # zeroed once; each call leaves it zeroed
         self._graph = None
 
