@@ -86,6 +86,11 @@ ATTN_CASES = {
     # G = 16 (Q by TMA, 8 nodes per 128-row group), a prefix ending inside a
     # page and a 256-node tree whose tiles fall into more than one split
     "g16_tree_cut": ([synth.budget_tree(np.random.default_rng(9), 256, 16, 8)], [2077], 16, 1, 128),
+    # 48 requests with prefixes from 16 to 1500 tokens and trees of 1 to 20
+    # nodes: 384 (request, KV head) units, so the launch takes one split per
+    # request and orders the units longest first
+    "lpt_48_ragged": ([synth.tiny_tree(np.random.default_rng(300 + i), 1 + (7 * i) % 20, 4, 3) for i in range(48)],
+                      [16 + (353 * i) % 1485 for i in range(48)], 16, 8, 64),
 }
 
 

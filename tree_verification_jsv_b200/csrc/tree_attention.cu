@@ -122,6 +122,83 @@ __device__ __forceinline__ int request_splits(int total, int C, int S) {
     return max(1, min(S, (total + C - 1) / C));
 }
 
+// Key tiles of a request: prefix tiles, then tree tiles from the page
+// boundary at or below P.
+__device__ __forceinline__ int request_tiles(const Request &r) {
+    return (r.P + kKeyTile - 1) / kKeyTile + (r.P + r.n - (r.P & ~15) + kKeyTile - 1) / kKeyTile;
+}
+
+// Longest-first order for batches of up to kLptMaxReqs requests (used when
+// the batch's largest request takes one split).  The CTAs
+// of a launch start in block order, so block L takes the L-th work unit
+// (request, KV head, row tile, split) with the requests sorted by tiles per
+// split, largest first (ties: lower request index first), and the blocks
+// past the last unit return at once: long units start first, short ones fill
+// the SMs as they free up, and no empty unit sits between them.  One warp
+// computes it from the request geometry; (b, unit index within b) or b = -1.
+constexpr int kLptMaxReqs = 64;
+
+__device__ __forceinline__ void lpt_unit(const AttnParams &prm, int L, int lane, int *s_units, int *s_b,
+                                         int &ub, int &uloc) {
+    const BatchArgs &a = prm.a;
+    const int G = a.Hq / a.Hkv;
+    int work[2], units[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int rb = lane + 32 * k;
+        work[k] = -1;
+        units[k] = 0;
+        Request q;
+        if (rb < a.B && load_request(a, rb, q)) {
+            const int K = request_tiles(q);
+            const int sb = request_splits(K, prm.C, prm.S);
+            units[k] = a.Hkv * ((q.n * G + kRowsPerCta - 1) / kRowsPerCta) * sb;
+            work[k] = (K + sb - 1) / sb;
+        }
+    }
+    int rank[2] = {0, 0};
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+        for (int j = 0; j < 32; ++j) {
+            const int wj = __shfl_sync(0xffffffffu, work[kk], j), bj = j + 32 * kk;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int bi = lane + 32 * k;
+                if (bj < a.B && (wj > work[k] || (wj == work[k] && bj < bi))) ++rank[k];
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        if (lane + 32 * k < a.B) {
+            s_units[rank[k]] = units[k];
+            s_b[rank[k]] = lane + 32 * k;
+        }
+    }
+    __syncwarp();
+    // exclusive prefix of the sorted units: lane l holds entries 2l, 2l + 1
+    const int e0 = 2 * lane, e1 = 2 * lane + 1;
+    const int u0 = e0 < a.B ? s_units[e0] : 0, u1 = e1 < a.B ? s_units[e1] : 0;
+    int incl = u0 + u1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    const int excl = incl - u0 - u1;
+    int fb = -1, fl = 0;
+    if (L >= excl && L < excl + u0) {
+        fb = s_b[e0];
+        fl = L - excl;
+    } else if (L >= excl + u0 && L < incl) {
+        fb = s_b[e1];
+        fl = L - excl - u0;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, fb >= 0);
+    ub = hit ? __shfl_sync(0xffffffffu, fb, __ffs(hit) - 1) : -1;
+    uloc = hit ? __shfl_sync(0xffffffffu, fl, __ffs(hit) - 1) : 0;
+}
+
 template <int D>
 struct AttnSmem {
     static constexpr int kQGroupBytes = kGroupRows * D * 2;    // one row group's Q
@@ -245,7 +322,10 @@ __device__ __forceinline__ void attention_mma_loop(uint32_t tmem, uint32_t aQ, u
     mbar_wait(drain_bar, 0, (volatile int *)&zero);
 }
 
-template <int D>
+// kLpt: the work unit comes from the longest-first order (batches of 2 to
+// kLptMaxReqs requests), else from the block index.  Two instantiations, so
+// that the second keeps the register allocation of a kernel without the order.
+template <int D, bool kLpt>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmQ, const AttnParams prm) {
@@ -263,14 +343,42 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     __shared__ int par_sh[32 * kMaxTreeWords];
 
     const BatchArgs &a = prm.a;
-    const int b = blockIdx.z / a.Hkv, g = blockIdx.z % a.Hkv;
     const int G = a.Hq / a.Hkv;
-    const int split = blockIdx.y;
-    const int m0 = blockIdx.x * kRowsPerCta;
-
-    // request geometry (uniform per CTA); invalid requests are flagged and skipped
+    // the work unit of this CTA: longest first for small ragged batches, else
+    // by block index (x: row tile, y: split, z: request x KV head)
+    int b, g, split, m0;
     Request r;
-    if (!load_request(a, b, r)) return;
+    if constexpr (kLpt) {
+        __shared__ int lpt_sh[2 * kLptMaxReqs + 2];
+        if (threadIdx.x < 32) {
+            const int L = (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+            int ub, uloc;
+            lpt_unit(prm, L, (int)threadIdx.x, lpt_sh, lpt_sh + kLptMaxReqs, ub, uloc);
+            if (threadIdx.x == 0) {
+                lpt_sh[2 * kLptMaxReqs] = ub;
+                lpt_sh[2 * kLptMaxReqs + 1] = uloc;
+            }
+        }
+        __syncthreads();
+        b = lpt_sh[2 * kLptMaxReqs];
+        if (b < 0 || !load_request(a, b, r)) return;
+        const int sb = request_splits(request_tiles(r), prm.C, prm.S);
+        const int R = (r.n * G + kRowsPerCta - 1) / kRowsPerCta;
+        // within a request: row tile fastest, then split, then KV head (the
+        // order of the block-index form, so that CTAs running side by side
+        // share K/V tiles in L2)
+        const int loc = lpt_sh[2 * kLptMaxReqs + 1];
+        m0 = (loc % R) * kRowsPerCta;
+        split = (loc / R) % sb;
+        g = loc / (R * sb);
+    } else {
+        b = blockIdx.z / a.Hkv;
+        g = blockIdx.z % a.Hkv;
+        split = blockIdx.y;
+        m0 = blockIdx.x * kRowsPerCta;
+        // request geometry (uniform per CTA); invalid requests are flagged and skipped
+        if (!load_request(a, b, r)) return;
+    }
     const int rows_total = r.n * G;
     if (m0 >= rows_total) return;
     const int rows_here = min(kRowsPerCta, rows_total - m0);
@@ -281,7 +389,7 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     // Sb splits, split s takes the balanced run [total * s / Sb, total * (s + 1) / Sb).
     const int prefix_tiles = (r.P + kKeyTile - 1) / kKeyTile;
     const int P0 = r.P & ~15;                    // tree tiles start on a page boundary
-    const int total_tiles = prefix_tiles + (r.P + r.n - P0 + kKeyTile - 1) / kKeyTile;
+    const int total_tiles = request_tiles(r);
     const int Sb = request_splits(total_tiles, prm.C, prm.S);
     if (split >= Sb) return;
     const int t_begin = (int)((long long)total_tiles * split / Sb);
@@ -688,52 +796,56 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         // slice of this group's Q buffer (free once the group's last product
         // has completed: every product of the group precedes its last PV), XOR-
         // swizzled by row so that neither side of the transpose has bank conflicts.
-        const bool direct = direct_sh != 0;
-        const float row_scale = direct ? (l > 0.f ? 1.f / l : 0.f) : 1.f;
         constexpr int kScrCols = D / 2;
         constexpr int kChunks = kScrCols / 4;                   // 16-byte chunks per staged row
         constexpr int kRowsPerStore = 32 / kChunks;
         float4 *scr = reinterpret_cast<float4 *>(sQ + grp * L::kQGroupBytes + sub * (32 * kScrCols * 4));
-        const long long my_off =
-            row_valid ? (long long)((direct ? row_id : (size_t)split * rows + row_id) * D) : -1ll;
         if (have_o) tc_fence_after();
+        // One pass stages half of D for the warp's 32 rows (scaled by `scale`)
+        // and hands each staged 16-byte chunk to `store(row offset, column, value)`.
+        auto write_rows = [&](long long my_off, float scale, auto store) {
 #pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
+            for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
-            for (int c0 = 0; c0 < kScrCols; c0 += 32) {
-                uint32_t rr[32];
-                if (have_o) {
-                    tmem_ld_32x32b_x32(tO + lane_addr + pass * kScrCols + c0, rr);   // warp-collective
-                    tmem_ld_wait();
-                } else {
+                for (int c0 = 0; c0 < kScrCols; c0 += 32) {
+                    uint32_t rr[32];
+                    if (have_o) {
+                        tmem_ld_32x32b_x32(tO + lane_addr + pass * kScrCols + c0, rr);   // warp-collective
+                        tmem_ld_wait();
+                    } else {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) rr[x] = 0u;
+                        for (int x = 0; x < 32; ++x) rr[x] = 0u;
+                    }
+#pragma unroll
+                    for (int x = 0; x < 8; ++x)
+                        scr[lane * kChunks + ((c0 / 4 + x) ^ (lane & (kChunks - 1)))] =
+                            make_float4(__uint_as_float(rr[4 * x]) * scale, __uint_as_float(rr[4 * x + 1]) * scale,
+                                        __uint_as_float(rr[4 * x + 2]) * scale, __uint_as_float(rr[4 * x + 3]) * scale);
                 }
-#pragma unroll
-                for (int x = 0; x < 8; ++x)
-                    scr[lane * kChunks + ((c0 / 4 + x) ^ (lane & (kChunks - 1)))] =
-                        make_float4(__uint_as_float(rr[4 * x]) * row_scale, __uint_as_float(rr[4 * x + 1]) * row_scale,
-                                    __uint_as_float(rr[4 * x + 2]) * row_scale,
-                                    __uint_as_float(rr[4 * x + 3]) * row_scale);
-            }
-            __syncwarp();
+                __syncwarp();
 #pragma unroll 4
-            for (int i = 0; i < 32; i += kRowsPerStore) {
-                const int wr = i + lane / kChunks, ch = lane % kChunks;
-                const long long off = __shfl_sync(0xffffffffu, my_off, wr);
-                const float4 v = scr[wr * kChunks + (ch ^ (wr & (kChunks - 1)))];
-                if (off < 0) continue;
-                if (direct)
-                    *reinterpret_cast<uint2 *>(prm.out + off + pass * kScrCols + ch * 4) =
-                        make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
-                else
-                    *reinterpret_cast<float4 *>(prm.ws_o + off + pass * kScrCols + ch * 4) = v;
+                for (int i = 0; i < 32; i += kRowsPerStore) {
+                    const int wr = i + lane / kChunks, ch = lane % kChunks;
+                    const long long off = __shfl_sync(0xffffffffu, my_off, wr);
+                    const float4 v = scr[wr * kChunks + (ch ^ (wr & (kChunks - 1)))];
+                    if (off >= 0) store(off + pass * kScrCols + ch * 4, v);
+                }
+                __syncwarp();
             }
-            __syncwarp();
-        }
-        if (row_valid && !direct) {
-            prm.ws_ml[((size_t)split * rows + row_id) * 2 + 0] = m_used;
-            prm.ws_ml[((size_t)split * rows + row_id) * 2 + 1] = l;
+        };
+        if (direct_sh) {
+            write_rows(row_valid ? (long long)(row_id * D) : -1ll, l > 0.f ? 1.f / l : 0.f,
+                       [&](long long o, const float4 &v) {
+                           *reinterpret_cast<uint2 *>(prm.out + o) = make_uint2(pack_bf16x2(v.x, v.y),
+                                                                                pack_bf16x2(v.z, v.w));
+                       });
+        } else {
+            write_rows(row_valid ? (long long)(((size_t)split * rows + row_id) * D) : -1ll, 1.f,
+                       [&](long long o, const float4 &v) { *reinterpret_cast<float4 *>(prm.ws_o + o) = v; });
+            if (row_valid) {
+                prm.ws_ml[((size_t)split * rows + row_id) * 2 + 0] = m_used;
+                prm.ws_ml[((size_t)split * rows + row_id) * 2 + 1] = l;
+            }
         }
     }
 
@@ -767,8 +879,7 @@ tree_attention_combine_kernel(BatchArgs a, int S_max, int C, const float *__rest
     Request r;
     if (!load_request(a, b, r)) return;
     if (rloc >= r.n * G) return;
-    const int total_tiles = (r.P + kKeyTile - 1) / kKeyTile + (r.P + r.n - (r.P & ~15) + kKeyTile - 1) / kKeyTile;
-    const int S = request_splits(total_tiles, C, S_max);
+    const int S = request_splits(request_tiles(r), C, S_max);
     if (S == 1) return;                              // the attention kernel wrote these rows
     const int i = rloc / G, h = g * G + rloc % G, t = r.base + i;
     const size_t row_id = (size_t)t * a.Hq + h;
@@ -886,21 +997,30 @@ static cudaError_t launch_d(const BatchArgs &a, const uint16_t *q, const uint16_
     if (!encode_tensor_map_3d(&tmV, v_cache, D, a.Hkv, slots, (uint64_t)D * 2, (uint64_t)a.Hkv * D * 2, 64, 1, 16))
         return cudaErrorInvalidValue;
     const size_t smem = (size_t)Lt::kTotal + 1024;
-    static PerDeviceOnce attr_once;
-    cudaError_t ae = attr_once.run([&]() {
-        cudaError_t e = cudaFuncSetAttribute(tree_attention_tc_kernel<D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto set_attrs = [&](auto kernel) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(tree_attention_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                      (int)cudaSharedmemCarveoutMaxShared);
         return e;
+    };
+    static PerDeviceOnce attr_once;
+    cudaError_t ae = attr_once.run([&]() {
+        cudaError_t e = set_attrs(tree_attention_tc_kernel<D, false>);
+        return e == cudaSuccess ? set_attrs(tree_attention_tc_kernel<D, true>) : e;
     });
     if (ae != cudaSuccess) return ae;
+    // Longest-first order when each CTA takes a request's whole key range
+    // (S = 1), so that the longest requests do not start last; with several
+    // splits the per-request split counts already even the units out, and the
+    // order's set-up and register cost is not paid.
+    const bool lpt = S == 1 && a.B > 1 && a.B <= kLptMaxReqs;
+    auto kernel = lpt ? tree_attention_tc_kernel<D, true> : tree_attention_tc_kernel<D, false>;
     dim3 grid((a.max_nodes * G + kRowsPerCta - 1) / kRowsPerCta, S, a.B * a.Hkv);
-    cudaError_t le = launch_pdl(tree_attention_tc_kernel<D>, grid, dim3(kAttnThreads), smem, st, tmK, tmV, tmQ, prm);
+    cudaError_t le = launch_pdl(kernel, grid, dim3(kAttnThreads), smem, st, tmK, tmV, tmQ, prm);
     if (le != cudaSuccess) {
         cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, tree_attention_tc_kernel<D>) == cudaSuccess)
+        if (cudaFuncGetAttributes(&fa, kernel) == cudaSuccess)
             note_launch_failure("tree attention", fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes,
                                 fa.maxDynamicSharedSizeBytes, kAttnThreads, smem);
         return le;
