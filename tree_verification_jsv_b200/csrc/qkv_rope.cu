@@ -27,6 +27,10 @@
 // to the first CTA through distributed shared memory (bounded mbarrier
 // handshakes: ready on the first CTA, free on the others), and the first CTA
 // adds them and runs the epilogue.
+// Under programmatic dependent launch the producer issues the first ring's
+// worth of W copies before it waits for the previous launch: W is a weight
+// that no call of this library writes, while x, the batch geometry and the
+// cache rows written here are read or written only after the wait.
 #include "jsv_internal.cuh"
 #include "sm100.cuh"
 
@@ -42,6 +46,9 @@ constexpr int kQTileM = 128;
 constexpr int kQKChunk = 64;
 constexpr uint32_t kQStageA = kQTileM * 128;
 constexpr int kQSmemBudget = 164 * 1024;
+// A smaller ring that lets two CTAs share an SM, so that clusters of three
+// find room in one resident wave (about 37 KB of static shared memory a CTA).
+constexpr int kQSmemBudgetShared = 72 * 1024;
 constexpr int kQMaxWalk = 512 + 256;             // parents a group's depth walks can visit
 
 struct QkvParams {
@@ -63,7 +70,6 @@ __global__ void __launch_bounds__(kQThreads, 1)
 qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                 const QkvParams p) {
     pdl_allow_dependents();
-    pdl_wait_predecessor();
     extern __shared__ uint8_t dsmem[];
     __shared__ __align__(8) uint64_t full_bar[kQMaxStages], empty_bar[kQMaxStages], accf_bar, drain_bar;
     __shared__ uint32_t tmem_base_sh;
@@ -108,6 +114,7 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
+    if (warp >= 2) pdl_wait_predecessor();       // the epilogue reads the geometry and writes q and the cache
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -115,10 +122,21 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             prefetch_tensormap(&tmW);
             prefetch_tensormap(&tmX);
             const uint32_t tx = kQStageA + (uint32_t)p.box_rows * 128;
-            int stage = 0;
-            uint32_t phase = 0;
-            long long issued = 0;
-            for (int kc = kc0; kc < kc1; ++kc) {
+            // the first ring's W copies (fresh stages need no wait), then the
+            // wait for the previous launch, then their x copies
+            const int npre = min(p.stages, kc1 - kc0);
+            for (int i = 0; i < npre; ++i) {
+                mbar_arrive_expect_tx(&full_bar[i], tx);
+                tma_load_2d(smem + (size_t)i * p.stage_bytes, &tmW, &full_bar[i], (kc0 + i) * kQKChunk, row0);
+            }
+            pdl_wait_predecessor();
+            for (int i = 0; i < npre; ++i)
+                tma_load_2d(smem + (size_t)i * p.stage_bytes + kQStageA, &tmX, &full_bar[i], (kc0 + i) * kQKChunk,
+                            node0);
+            int stage = npre == p.stages ? 0 : npre;
+            uint32_t phase = npre == p.stages ? 1u : 0u;
+            long long issued = npre;
+            for (int kc = kc0 + npre; kc < kc1; ++kc) {
                 if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh)) {
                     abort_sh = 1;
                     flag_error(a.dev_status, JSV_ERR_TIMEOUT);
@@ -348,8 +366,8 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
     p.group_nodes = a.total_nodes <= 256 ? ((a.total_nodes + 15) & ~15) : 256;
     p.box_rows = p.group_nodes;
     p.stage_bytes = kQStageA + (uint32_t)p.box_rows * 128;
-    p.stages = kQSmemBudget / (int)p.stage_bytes;
-    if (p.stages > kQMaxStages) p.stages = kQMaxStages;
+    auto stages_for = [&](int budget) { return min(kQMaxStages, budget / (int)p.stage_bytes); };
+    p.stages = stages_for(kQSmemBudget);
     p.cos = rope_cos;
     p.sin = rope_sin;
     p.max_pos = max_pos;
@@ -363,7 +381,7 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
         return cudaErrorInvalidValue;
     if (!encode_tensor_map_2d(&tmX, x, (uint64_t)d, (uint64_t)a.total_nodes, (uint64_t)d * 2, kQKChunk, p.box_rows))
         return cudaErrorInvalidValue;
-    const size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
+    size_t smem = (size_t)p.stages * p.stage_bytes + 1024;
     static PerDeviceOnce attr_once;
     cudaError_t ae = attr_once.run([]() {
         cudaError_t e = cudaFuncSetAttribute(qkv_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -378,29 +396,44 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
     const int groups = (a.total_nodes + p.group_nodes - 1) / p.group_nodes;
     // Too few (tile, group) CTAs to stream the weight with every SM: split K
     // over a cluster of up to four CTAs (each keeping at least four chunks),
-    // as many as the SMs and the resident clusters allow.
+    // as many as the SMs and the resident clusters allow.  Clusters are placed
+    // within one GPC, so a split that does not fit in one wave with the full
+    // ring is tried again with the smaller ring, which lets two CTAs share an
+    // SM; more CTAs streaming W beat a deeper ring per CTA.
     const int sms = device_sm_count();
     int ks = 1;
     while (ks < 4 && (long long)tiles * groups * (ks + 1) <= sms && p.kchunks / (ks + 1) >= 4) ++ks;
-    for (; ks > 1; --ks) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(tiles * ks, groups);
-        cfg.blockDim = dim3(kQThreads);
-        cfg.dynamicSmemBytes = smem;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = ks;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, qkv_rope_kernel, &cfg) != cudaSuccess) {
-            cudaGetLastError();
-            n = 0;
+    bool placed = false;
+    for (; ks > 1 && !placed; --ks) {
+        for (int budget : {kQSmemBudget, kQSmemBudgetShared}) {
+            const int st_n = stages_for(budget);
+            if (st_n < 2) continue;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(tiles * ks, groups);
+            cfg.blockDim = dim3(kQThreads);
+            cfg.dynamicSmemBytes = (size_t)st_n * p.stage_bytes + 1024;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = ks;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, qkv_rope_kernel, &cfg) != cudaSuccess) {
+                cudaGetLastError();
+                n = 0;
+            }
+            if ((long long)n >= (long long)tiles * groups) {     // one resident wave
+                p.stages = st_n;
+                smem = cfg.dynamicSmemBytes;
+                placed = true;
+                break;
+            }
         }
-        if ((long long)n >= (long long)tiles * groups) break;     // one resident wave
+        if (placed) break;
     }
+    if (!placed) ks = 1;
     p.ksplit = ks;
     dim3 grid(tiles * ks, groups);
     cudaError_t e = ks > 1 ? launch_pdl_cluster(qkv_rope_kernel, grid, dim3(kQThreads), smem, st, ks, tmW, tmX, p)
