@@ -62,7 +62,11 @@ typedef enum {
     JSV_ERR_UNSUPPORTED = 2,   /* shape outside the supported set            */
     JSV_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed       */
     JSV_ERR_TIMEOUT = 4,       /* a bounded device wait gave up              */
-    JSV_ERR_DEVICE_INPUT = 5   /* written to *dev_status: bad device data    */
+    JSV_ERR_DEVICE_INPUT = 5,  /* written to *dev_status: bad device data    */
+    JSV_ERR_BOUNDS = 6         /* written to *dev_status, only by a library
+                                  built with JSV_CHECK_BOUNDS: a computed
+                                  index fell outside its buffer (a library
+                                  fault; the access was skipped)            */
 } jsv_status;
 
 /*
@@ -346,6 +350,13 @@ JSV_API const char *jsv_status_string(jsv_status status);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 JSV_API int32_t jsv_version(void);
+
+/* Build flags of this library: bit 0 set when it was compiled with
+ * JSV_CHECK_BOUNDS (libjsv_checked.so), i.e. every computed global index
+ * of the kernels is compared with its buffer's extent before the access and
+ * a miss is skipped and written to the status word as JSV_ERR_BOUNDS.  The
+ * pages have no counterpart: it is a debugging aid of this library. */
+JSV_API int32_t jsv_build_flags(void);
 
 #ifdef __cplusplus
 }

@@ -107,3 +107,17 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(jsv, "_lib", None)
     with pytest.raises(RuntimeError):
         jsv.load()
+
+
+def test_checked_build_exports_the_same_symbols_and_says_so(lib):
+    """libjsv_checked.so (-DJSV_CHECK_BOUNDS) exports every declared symbol
+    and reports its build flag; the ordinary library reports none."""
+    so = jbuild.build(checked=True)
+    chk = ctypes.CDLL(str(so))
+    for n in declared_symbols():
+        assert hasattr(chk, n), n
+    chk.jsv_build_flags.restype = ctypes.c_int32
+    assert chk.jsv_build_flags() & 1 == 1
+    assert jsv.jsv_build_flags() & 1 == 0
+    chk.jsv_status_string.restype = ctypes.c_char_p
+    assert b"bounds" in chk.jsv_status_string(jsv.JSV_ERR_BOUNDS)

@@ -168,11 +168,20 @@ const char *jsv_status_string(jsv_status status) {
         case JSV_ERR_CUDA: return "CUDA error";
         case JSV_ERR_TIMEOUT: return "device wait timed out";
         case JSV_ERR_DEVICE_INPUT: return "malformed device-side input";
+        case JSV_ERR_BOUNDS: return "index out of bounds (checked build)";
     }
     return "unknown status";
 }
 
 int32_t jsv_version(void) { return 100; }
+
+int32_t jsv_build_flags(void) {
+#ifdef JSV_CHECK_BOUNDS
+    return 1;
+#else
+    return 0;
+#endif
+}
 
 const char *jsv_last_error_string(void) {
     static thread_local char buf[512];

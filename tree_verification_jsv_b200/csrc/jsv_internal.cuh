@@ -88,6 +88,23 @@ __device__ __forceinline__ void flag_error(int32_t *status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// Index checks of the checked build (-DJSV_CHECK_BOUNDS, libjsv_checked.so):
+// a computed global index is compared with its buffer's extent before the
+// access, and one outside records JSV_ERR_BOUNDS in the status word and the
+// access is skipped.  The kernels' own input checks keep every index in
+// range, so a failure here is a fault of the library.  In the ordinary
+// build the check is `true` and costs nothing.
+#ifdef JSV_CHECK_BOUNDS
+__device__ __forceinline__ bool index_ok(long long i, long long n, int32_t *status) {
+    if (i >= 0 && i < n) return true;
+    flag_error(status, JSV_ERR_BOUNDS);
+    return false;
+}
+#define JSV_IN_BOUNDS(i, n, status) ::jsv::index_ok((long long)(i), (long long)(n), (status))
+#else
+#define JSV_IN_BOUNDS(i, n, status) ((void)(i), (void)(n), true)
+#endif
+
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
     return __uint_as_float(((uint32_t)h) << 16);
 }
@@ -100,6 +117,7 @@ struct Request {
 };
 
 __device__ __forceinline__ bool load_request(const BatchArgs &a, int b, Request &r) {
+    if (!JSV_IN_BOUNDS(b, a.B, a.dev_status)) return false;
     int s = a.node_offsets[b], e = a.node_offsets[b + 1];
     int P = a.prefix_len[b];
     bool ok = s >= 0 && e > s && e <= a.total_nodes && (e - s) <= a.max_nodes &&
@@ -117,7 +135,9 @@ __device__ __forceinline__ bool load_request(const BatchArgs &a, int b, Request 
 // Physical row index (page * page_size + offset) of logical slot s, or -1
 // (flagged) if the page entry is out of range.
 __device__ __forceinline__ long long slot_phys_row(const BatchArgs &a, int b, int s) {
-    int page = a.page_table[(size_t)b * a.max_pages_per_req + s / a.page_size];
+    const long long pi = (long long)b * a.max_pages_per_req + s / a.page_size;
+    if (!JSV_IN_BOUNDS(pi, (long long)a.B * a.max_pages_per_req, a.dev_status)) return -1;
+    int page = a.page_table[pi];
     if (page < 0 || page >= a.num_pages) {
         flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
         return -1;

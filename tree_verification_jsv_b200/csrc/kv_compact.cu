@@ -29,6 +29,7 @@ __device__ void compact_rows(const BatchArgs &a, int b, const Request &r, const 
                              uint16_t *cache, int h0, int heads, uint4 *stage, int *s_src, int *s_dst) {
     const int vec_per_head = a.D / 8;
     const int vec_per_row = heads * vec_per_head;
+    const long long cache_elems = (long long)a.num_pages * a.page_size * a.Hkv * a.D;
     for (int k0 = 0; k0 <= acc; k0 += kCompactChunk) {
         const int rows = min(kCompactChunk, acc + 1 - k0);
         for (int i = threadIdx.x; i < rows; i += blockDim.x) {
@@ -40,17 +41,20 @@ __device__ void compact_rows(const BatchArgs &a, int b, const Request &r, const 
             const int i = e / vec_per_row, c = e % vec_per_row;
             const int hh = c / vec_per_head, x = c % vec_per_head;
             if (s_src[i] == s_dst[i]) continue;
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                cache + ((size_t)s_src[i] * a.Hkv + h0 + hh) * a.D);
-            stage[e] = src[x];
+            const long long si = ((long long)s_src[i] * a.Hkv + h0 + hh) * a.D + x * 8;
+            if (!JSV_IN_BOUNDS(si + 7, cache_elems, a.dev_status) || !JSV_IN_BOUNDS(si, cache_elems, a.dev_status))
+                continue;
+            stage[e] = *reinterpret_cast<const uint4 *>(cache + si);
         }
         __syncthreads();
         for (int e = threadIdx.x; e < rows * vec_per_row; e += blockDim.x) {
             const int i = e / vec_per_row, c = e % vec_per_row;
             const int hh = c / vec_per_head, x = c % vec_per_head;
             if (s_src[i] == s_dst[i]) continue;
-            uint4 *dst = reinterpret_cast<uint4 *>(cache + ((size_t)s_dst[i] * a.Hkv + h0 + hh) * a.D);
-            dst[x] = stage[e];
+            const long long di = ((long long)s_dst[i] * a.Hkv + h0 + hh) * a.D + x * 8;
+            if (!JSV_IN_BOUNDS(di + 7, cache_elems, a.dev_status) || !JSV_IN_BOUNDS(di, cache_elems, a.dev_status))
+                continue;
+            *reinterpret_cast<uint4 *>(cache + di) = stage[e];
         }
         __syncthreads();
     }

@@ -224,7 +224,9 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 bool ok = true;
                 while (j > 0) {
                     const int gi = req.base + j;
-                    const int pj = (staged && gi >= wbase && gi < wbase + wcount) ? s_par[gi - wbase] : a.parent[gi];
+                    int pj = -1;
+                    if (staged && gi >= wbase && gi < wbase + wcount) pj = s_par[gi - wbase];
+                    else if (JSV_IN_BOUNDS(gi, a.total_nodes, a.dev_status)) pj = a.parent[gi];
                     if (pj < 0 || pj >= j || ++steps > req.n) { ok = false; break; }
                     j = pj;
                     ++dep;
@@ -309,7 +311,8 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         const int pos = c < in_group ? s_pos[c] : -1;
                         cs[k] = make_float4(1.f, 1.f, 1.f, 1.f);
                         sn[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (kq < 2 && qvalid && pos >= 0) {
+                        if (kq < 2 && qvalid && pos >= 0 &&
+                            JSV_IN_BOUNDS((long long)pos * half + iq + 3, (long long)p.max_pos * half, a.dev_status)) {
                             cs[k] = __ldg(reinterpret_cast<const float4 *>(p.cos + (size_t)pos * half + iq));
                             sn[k] = __ldg(reinterpret_cast<const float4 *>(p.sin + (size_t)pos * half + iq));
                         }
@@ -333,8 +336,12 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         pk.x = (uint32_t)to_bf16_bits(v.x) | ((uint32_t)to_bf16_bits(v.y) << 16);
                         pk.y = (uint32_t)to_bf16_bits(v.z) | ((uint32_t)to_bf16_bits(v.w) << 16);
                         const int t = node0 + c;
-                        uint16_t *dst = kq == 0 ? p.q + ((size_t)t * a.Hq + headq) * a.D + oq
-                                        : (kq == 1 ? p.k_cache : p.v_cache) + ((size_t)prow * a.Hkv + headq) * a.D + oq;
+                        const long long di = kq == 0 ? ((long long)t * a.Hq + headq) * a.D + oq
+                                                     : ((long long)prow * a.Hkv + headq) * a.D + oq;
+                        const long long dn = kq == 0 ? (long long)a.total_nodes * a.Hq * a.D
+                                                     : (long long)a.num_pages * a.page_size * a.Hkv * a.D;
+                        if (!JSV_IN_BOUNDS(di + 3, dn, a.dev_status)) continue;
+                        uint16_t *dst = (kq == 0 ? p.q : (kq == 1 ? p.k_cache : p.v_cache)) + di;
                         *reinterpret_cast<uint2 *>(dst) = pk;
                     }
                 }

@@ -473,7 +473,9 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 int page = -2;
                 if (lane < kKeyTile / 16) {
                     const int lp = tile_slot0(j) / 16 + lane;
-                    if (lp < mapped_pages) page = __ldg(a.page_table + (size_t)b * a.max_pages_per_req + lp);
+                    const long long pi = (long long)b * a.max_pages_per_req + lp;
+                    if (lp < mapped_pages && JSV_IN_BOUNDS(pi, (long long)a.B * a.max_pages_per_req, a.dev_status))
+                        page = __ldg(a.page_table + pi);
                 }
                 return page;
             };
@@ -595,7 +597,8 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 #pragma unroll
             for (int it = 0; it < kParIters; ++it) {
                 const int i = et + it * (kGroups * 128);
-                pv[it] = i < r.n ? __ldg(a.parent + r.base + i) : -1;
+                pv[it] = (i < r.n && JSV_IN_BOUNDS(r.base + i, a.total_nodes, a.dev_status))
+                             ? __ldg(a.parent + r.base + i) : -1;
             }
         }
         if (!prm.q_tma) {
@@ -611,9 +614,9 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     qv[it] = make_uint4(0, 0, 0, 0);
                     if (rr < rows_here) {
                         const int rgg = m0 + rr;
-                        const uint16_t *src =
-                            prm.q + ((size_t)(r.base + rgg / G) * a.Hq + g * G + rgg % G) * D + c * 8;
-                        qv[it] = __ldg(reinterpret_cast<const uint4 *>(src));
+                        const size_t qi = ((size_t)(r.base + rgg / G) * a.Hq + g * G + rgg % G) * D + c * 8;
+                        if (JSV_IN_BOUNDS(qi + 7, (long long)a.total_nodes * a.Hq * D, a.dev_status))
+                            qv[it] = __ldg(reinterpret_cast<const uint4 *>(prm.q + qi));
                     }
                 }
 #pragma unroll
@@ -836,15 +839,20 @@ tree_attention_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         if (direct_sh) {
             write_rows(row_valid ? (long long)(row_id * D) : -1ll, l > 0.f ? 1.f / l : 0.f,
                        [&](long long o, const float4 &v) {
-                           *reinterpret_cast<uint2 *>(prm.out + o) = make_uint2(pack_bf16x2(v.x, v.y),
-                                                                                pack_bf16x2(v.z, v.w));
+                           if (JSV_IN_BOUNDS(o + 3, (long long)rows * D, a.dev_status))
+                               *reinterpret_cast<uint2 *>(prm.out + o) = make_uint2(pack_bf16x2(v.x, v.y),
+                                                                                    pack_bf16x2(v.z, v.w));
                        });
         } else {
             write_rows(row_valid ? (long long)(((size_t)split * rows + row_id) * D) : -1ll, 1.f,
-                       [&](long long o, const float4 &v) { *reinterpret_cast<float4 *>(prm.ws_o + o) = v; });
-            if (row_valid) {
-                prm.ws_ml[((size_t)split * rows + row_id) * 2 + 0] = m_used;
-                prm.ws_ml[((size_t)split * rows + row_id) * 2 + 1] = l;
+                       [&](long long o, const float4 &v) {
+                           if (JSV_IN_BOUNDS(o + 3, (long long)prm.S * rows * D, a.dev_status))
+                               *reinterpret_cast<float4 *>(prm.ws_o + o) = v;
+                       });
+            const size_t mi = ((size_t)split * rows + row_id) * 2;
+            if (row_valid && JSV_IN_BOUNDS(mi + 1, (long long)prm.S * rows * 2, a.dev_status)) {
+                prm.ws_ml[mi + 0] = m_used;
+                prm.ws_ml[mi + 1] = l;
             }
         }
     }
@@ -887,6 +895,7 @@ tree_attention_combine_kernel(BatchArgs a, int S_max, int C, const float *__rest
     // lane s holds split s's (max, sum); the merge weights come from warp
     // reductions, so the partial loads below are independent of each other
     float ms = -INFINITY, ls = 0.f;
+    if (!JSV_IN_BOUNDS(row_id, rows, a.dev_status) || !JSV_IN_BOUNDS(S - 1, S_max, a.dev_status)) return;
     if (lane < S) {
         const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + ((size_t)lane * rows + row_id) * 2);
         ms = ml.x;

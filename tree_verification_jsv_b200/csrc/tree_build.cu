@@ -253,8 +253,9 @@ accum_logp_tree_kernel(TreeArgs a) {
             const int d = sm.ndepth[i];
             o_par[i] = sm.nparent[i];
             o_dep[i] = d;
+            const long long ti = (((long long)b * a.D) + (d - 1)) * k + sm.nrank[i];
             o_tok[i] = d == 0 ? a.root_token[b]
-                              : a.topk_tokens[(((size_t)b * a.D) + (d - 1)) * k + sm.nrank[i]];
+                       : (JSV_IN_BOUNDS(ti, (long long)a.B * a.D * k, a.status) ? a.topk_tokens[ti] : -1);
             if (o_sc) o_sc[i] = sm.nscore[i];
         } else {
             o_par[i] = -1;

@@ -4,13 +4,19 @@ Every function has the name of the C entry point it calls (``include/jsv.h``)
 and takes torch tensors (or raw integer device addresses).  There is no
 fallback: if ``libjsv.so`` is missing or fails to load, every call raises.
 Build it with ``python -m tree_verification_jsv_b200.build``.
+
+With ``JSV_LIBRARY=checked`` in the environment the binding loads the
+checked build, ``libjsv_checked.so`` (every computed global index checked,
+misses reported as JSV_ERR_BOUNDS), from the same directory instead.
 """
 from __future__ import annotations
 
 import ctypes
+import os
 from pathlib import Path
 
-_SO = Path(__file__).resolve().parent / "libjsv.so"
+_DIR = Path(__file__).resolve().parent
+_SO = _DIR / ("libjsv_checked.so" if os.environ.get("JSV_LIBRARY") == "checked" else "libjsv.so")
 _lib = None
 
 JSV_OK = 0
@@ -19,13 +25,14 @@ JSV_ERR_UNSUPPORTED = 2
 JSV_ERR_CUDA = 3
 JSV_ERR_TIMEOUT = 4
 JSV_ERR_DEVICE_INPUT = 5
+JSV_ERR_BOUNDS = 6
 
 EXPORTS = ("jsv_tree_attention_workspace_size", "jsv_tree_attention",
            "jsv_lmhead_argmax_workspace_size", "jsv_lmhead_argmax", "jsv_accept_path",
            "jsv_kv_compact", "jsv_status_string", "jsv_version", "jsv_kernel_launches",
            "jsv_lmhead_argmax_noalloc", "jsv_last_error_string", "jsv_selftest_wait_timeout",
            "jsv_selftest_lmhead_timeout",
-           "jsv_accum_logp_tree", "jsv_tree_qkv_rope", "jsv_accept_compact")
+           "jsv_accum_logp_tree", "jsv_tree_qkv_rope", "jsv_accept_compact", "jsv_build_flags")
 
 # Largest node count jsv_lmhead_argmax_noalloc accepts (JSV_NOALLOC_MAX_NODES).
 NOALLOC_MAX_NODES = 8192
@@ -61,7 +68,7 @@ def load() -> ctypes.CDLL:
     if _lib is not None:
         return _lib
     if not _SO.exists():
-        raise RuntimeError(f"libjsv.so not built at {_SO}; run python -m tree_verification_jsv_b200.build")
+        raise RuntimeError(f"{_SO.name} not built at {_SO}; run python -m tree_verification_jsv_b200.build")
     lib = ctypes.CDLL(str(_SO))
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     bp = ctypes.POINTER(jsv_batch)
@@ -83,6 +90,8 @@ def load() -> ctypes.CDLL:
     lib.jsv_status_string.restype = ctypes.c_char_p
     lib.jsv_version.argtypes = []
     lib.jsv_version.restype = i32
+    lib.jsv_build_flags.argtypes = []
+    lib.jsv_build_flags.restype = i32
     lib.jsv_lmhead_argmax_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp, vp, vp]
     lib.jsv_lmhead_argmax_noalloc.restype = ctypes.c_int
     lib.jsv_tree_qkv_rope.argtypes = [bp, vp, vp, i32, vp, vp, i32, vp, vp, vp, vp]
@@ -129,6 +138,11 @@ def status_string(status: int) -> str:
 
 def jsv_version() -> int:
     return int(load().jsv_version())
+
+
+def jsv_build_flags() -> int:
+    """Bit 0: the loaded library is the checked build (JSV_CHECK_BOUNDS)."""
+    return int(load().jsv_build_flags())
 
 
 def jsv_kernel_launches() -> int:
