@@ -15,6 +15,7 @@ accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
     __shared__ int32_t s_par[kWalkWarps][kWalkMaxNodes];
     __shared__ int32_t s_tok[kWalkWarps][kWalkMaxNodes];
     __shared__ int32_t s_arg[kWalkWarps][kWalkMaxNodes];
+    __shared__ int32_t s_next[kWalkWarps][kWalkMaxNodes];
     const int w = threadIdx.x >> 5;
     const int b = blockIdx.x * kWalkWarps + w;
     const int lane = threadIdx.x & 31;
@@ -46,7 +47,7 @@ accept_path_kernel(BatchArgs a, const int32_t *__restrict__ tokens,
 
     int last = 0;
     bool cut = false;
-    const int len = greedy_walk_warp(s_par[w], s_tok[w], s_arg[w], r.n, max_path, row, lane, last, cut);
+    const int len = greedy_walk_warp(s_par[w], s_tok[w], s_arg[w], s_next[w], r.n, max_path, row, lane, last, cut);
     if (cut && lane == 0) flag_error(a.dev_status, JSV_ERR_DEVICE_INPUT);
     if (lane == 0) {
         row[0] = 0;

@@ -21,20 +21,27 @@ constexpr int kCompactThreads = 256;
 constexpr int kCompactChunk = 64;        // rows per chunk
 constexpr int kHeadsPerCta = 2;
 
+// Page entries of the tree's slots P .. P + n - 1 (pages P/16 .. (P+n-1)/16),
+// staged by the validation pass so that the move needs no page-table loads.
+constexpr int kTreePages = 40;           // (n - 1)/16 + 2 for n <= 512
+
 // Moves rows k = 0..acc (slot P + path[k] -> slot P + k) of KV heads
 // [h0, h0 + heads) of one cache, in chunks of increasing k; inside a chunk
 // every source is read into shared memory before any destination is written.
+// `s_pages` holds the checked entries of the tree's pages from page pg0 on.
 // Every thread of the block calls it.
-__device__ void compact_rows(const BatchArgs &a, int b, const Request &r, const int32_t *pathrow, int acc,
-                             uint16_t *cache, int h0, int heads, uint4 *stage, int *s_src, int *s_dst) {
+__device__ void compact_rows(const BatchArgs &a, const Request &r, const int32_t *pathrow, int acc,
+                             uint16_t *cache, int h0, int heads, uint4 *stage, int *s_src, int *s_dst,
+                             const int32_t *s_pages, int pg0) {
     const int vec_per_head = a.D / 8;
     const int vec_per_row = heads * vec_per_head;
     const long long cache_elems = (long long)a.num_pages * a.page_size * a.Hkv * a.D;
+    auto phys = [&](int slot) { return s_pages[slot / a.page_size - pg0] * a.page_size + slot % a.page_size; };
     for (int k0 = 0; k0 <= acc; k0 += kCompactChunk) {
         const int rows = min(kCompactChunk, acc + 1 - k0);
         for (int i = threadIdx.x; i < rows; i += blockDim.x) {
-            s_src[i] = (int)slot_phys_row(a, b, r.P + pathrow[k0 + i]);
-            s_dst[i] = (int)slot_phys_row(a, b, r.P + k0 + i);
+            s_src[i] = phys(r.P + pathrow[k0 + i]);
+            s_dst[i] = phys(r.P + k0 + i);
         }
         __syncthreads();
         for (int e = threadIdx.x; e < rows * vec_per_row; e += blockDim.x) {
@@ -60,6 +67,20 @@ __device__ void compact_rows(const BatchArgs &a, int b, const Request &r, const 
     }
 }
 
+// Loads the page entries of the tree's slots (pages P/16 .. (P+n-1)/16) into
+// s_pages, spread over the block; returns 1 if any is outside [0, num_pages).
+__device__ __forceinline__ int stage_tree_pages(const BatchArgs &a, int b, const Request &r, int32_t *s_pages) {
+    const int pg0 = r.P / a.page_size, pg1 = (r.P + r.n - 1) / a.page_size;
+    int bad = 0;
+    for (int pg = pg0 + threadIdx.x; pg <= pg1; pg += blockDim.x) {
+        const long long pi = (long long)b * a.max_pages_per_req + pg;
+        const int page = JSV_IN_BOUNDS(pi, (long long)a.B * a.max_pages_per_req, a.dev_status) ? a.page_table[pi] : -1;
+        if (page < 0 || page >= a.num_pages) bad = 1;
+        s_pages[pg - pg0] = page;
+    }
+    return bad;
+}
+
 __global__ void __launch_bounds__(kCompactThreads)
 kv_compact_kernel(BatchArgs a, uint16_t *__restrict__ k_cache, uint16_t *__restrict__ v_cache,
                   const int32_t *__restrict__ path, int max_path,
@@ -68,6 +89,7 @@ kv_compact_kernel(BatchArgs a, uint16_t *__restrict__ k_cache, uint16_t *__restr
     pdl_wait_predecessor();
     extern __shared__ uint4 stage[];      // [kCompactChunk][heads][D/8]
     __shared__ int s_src[kCompactChunk], s_dst[kCompactChunk];
+    __shared__ int32_t s_pages[kTreePages];
     const int b = blockIdx.x;
     uint16_t *cache = blockIdx.y == 0 ? k_cache : v_cache;
     const int h0 = blockIdx.z * kHeadsPerCta;
@@ -80,16 +102,13 @@ kv_compact_kernel(BatchArgs a, uint16_t *__restrict__ k_cache, uint16_t *__restr
     const int acc = req_ok ? accept_len[b] : 0;
     int bad = !req_ok || acc < 0 || acc >= r.n || acc + 1 > max_path;
     const int32_t *row = path + (size_t)b * max_path;
+    const int pg0 = req_ok ? r.P / a.page_size : 0;
     if (!bad) {
         for (int k = threadIdx.x; k <= acc; k += blockDim.x) {
             const int pk = row[k];
             if (k == 0 ? pk != 0 : (pk <= row[k - 1] || pk >= r.n)) bad = 1;
         }
-        const int pg0 = r.P / a.page_size, pg1 = (r.P + r.n - 1) / a.page_size;
-        for (int pg = pg0 + threadIdx.x; pg <= pg1; pg += blockDim.x) {
-            const int page = a.page_table[(size_t)b * a.max_pages_per_req + pg];
-            if (page < 0 || page >= a.num_pages) bad = 1;
-        }
+        bad |= stage_tree_pages(a, b, r, s_pages);
     }
     bad = __syncthreads_or(bad);
     if (bad) {
@@ -98,7 +117,7 @@ kv_compact_kernel(BatchArgs a, uint16_t *__restrict__ k_cache, uint16_t *__restr
     }
     if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) new_len[b] = r.P + acc + 1;
 
-    compact_rows(a, b, r, row, acc, cache, h0, heads, stage, s_src, s_dst);
+    compact_rows(a, r, row, acc, cache, h0, heads, stage, s_src, s_dst, s_pages, pg0);
 }
 
 // ---------------------------------------------------------------------------
@@ -118,6 +137,7 @@ accept_compact_kernel(BatchArgs a, const int32_t *__restrict__ tokens, const int
     extern __shared__ uint4 stage[];      // [kCompactChunk][heads][D/8]
     __shared__ int s_src[kCompactChunk], s_dst[kCompactChunk];
     __shared__ int32_t s_par[kWalkMaxNodes], s_tok[kWalkMaxNodes], s_arg[kWalkMaxNodes], s_path[kWalkMaxNodes];
+    __shared__ int32_t s_next[kWalkMaxNodes], s_pages[kTreePages];
     __shared__ int s_len, s_last;
     const int b = blockIdx.x;
     const bool writer = blockIdx.y == 0 && blockIdx.z == 0;
@@ -135,14 +155,8 @@ accept_compact_kernel(BatchArgs a, const int32_t *__restrict__ tokens, const int
     Request r;
     const bool req_ok = load_request(a, b, r) && r.n <= kWalkMaxNodes;
     int par_bad = 0, bad = 0;
-    if (req_ok) {
-        // every page the move touches must be mapped (the compaction's check)
-        const int pg0 = r.P / a.page_size, pg1 = (r.P + r.n - 1) / a.page_size;
-        for (int pg = pg0 + threadIdx.x; pg <= pg1; pg += blockDim.x) {
-            const int page = a.page_table[(size_t)b * a.max_pages_per_req + pg];
-            if (page < 0 || page >= a.num_pages) bad = 1;
-        }
-    }
+    const int pg0 = req_ok ? r.P / a.page_size : 0;
+    if (req_ok) bad = stage_tree_pages(a, b, r, s_pages);   // every page the move touches must be mapped
     if (req_ok) {
         for (int j = threadIdx.x; j < r.n; j += blockDim.x) {
             const int p = a.parent[r.base + j];
@@ -172,7 +186,7 @@ accept_compact_kernel(BatchArgs a, const int32_t *__restrict__ tokens, const int
         if (warp == 0) {
             int last = 0;
             bool cut = false;
-            const int len = greedy_walk_warp(s_par, s_tok, s_arg, r.n, max_path, s_path, lane, last, cut);
+            const int len = greedy_walk_warp(s_par, s_tok, s_arg, s_next, r.n, max_path, s_path, lane, last, cut);
             if (lane == 0) {
                 s_path[0] = 0;
                 s_len = len;
@@ -199,7 +213,7 @@ accept_compact_kernel(BatchArgs a, const int32_t *__restrict__ tokens, const int
     }
     if (threadIdx.x == 0 && writer) new_len[b] = r.P + acc + 1;
 
-    compact_rows(a, b, r, s_path, acc, cache, h0, heads, stage, s_src, s_dst);
+    compact_rows(a, r, s_path, acc, cache, h0, heads, stage, s_src, s_dst, s_pages, pg0);
 }
 
 cudaError_t launch_kv_compact(const BatchArgs &a, uint16_t *k_cache, uint16_t *v_cache,

@@ -6,9 +6,10 @@
 // target's own logits, so decoding is lossless.  At temperature 0 that is
 // the greedy descent: from the root, step to the smallest-index child whose
 // draft token equals the target's argmax at the current node, until no
-// child matches.  Children have larger indices than their parent
-// (topological order), so each step scans indices > cur with a warp ballot
-// and takes the lowest set lane of the first chunk that has a match.
+// child matches.  One pass over the nodes, a node per lane, records for
+// every node the smallest index of a child whose draft token equals the
+// node's argmax (a shared-memory atomicMin); the walk then follows these
+// links from the root, one shared-memory load per accepted token.
 #pragma once
 
 #include "jsv_internal.cuh"
@@ -17,32 +18,34 @@ namespace jsv {
 
 constexpr int kWalkMaxNodes = 512;
 
-// Walks the tree of n nodes; lane 0 writes path entries 1, 2, ... to `out`
-// (entry 0 is the root and is the caller's).  Returns the path length, root
-// included; `last` receives the last accepted node and `cut` is set when a
-// further match would make the path longer than max_path (the walk stops
-// there).  Every lane of the warp must call it.
+// Walks the tree of n nodes (parents already checked: 0 <= parent[j] < j
+// for j > 0); lane 0 writes path entries 1, 2, ... to `out` (entry 0 is the
+// root and is the caller's).  `s_next` is [n] shared scratch.  Returns the
+// path length, root included; `last` receives the last accepted node and
+// `cut` is set when a further match would make the path longer than
+// max_path (the walk stops there).  Every lane of the warp must call it.
 __device__ __forceinline__ int greedy_walk_warp(const int32_t *s_par, const int32_t *s_tok, const int32_t *s_arg,
-                                                int n, int max_path, int32_t *out, int lane, int &last, bool &cut) {
+                                                int32_t *s_next, int n, int max_path, int32_t *out, int lane,
+                                                int &last, bool &cut) {
+    for (int j = lane; j < n; j += 32) s_next[j] = n;          // no accepted child
+    __syncwarp();
+    for (int j = 1 + lane; j < n; j += 32) {
+        const int p = s_par[j];
+        if (s_tok[j] == s_arg[p]) atomicMin(&s_next[p], j);
+    }
+    __syncwarp();
     int cur = 0, len = 1;
     cut = false;
     while (true) {
-        const int want = s_arg[cur];
-        int found = -1;
-        for (int j0 = cur + 1; j0 < n; j0 += 32) {
-            const int j = j0 + lane;
-            const bool m = j < n && s_par[j] == cur && s_tok[j] == want;
-            const unsigned bal = __ballot_sync(0xffffffffu, m);
-            if (bal) { found = j0 + __ffs(bal) - 1; break; }
-        }
-        if (found < 0) break;
+        const int nx = s_next[cur];
+        if (nx >= n) break;
         if (len >= max_path) {
             cut = true;
             break;
         }
-        if (lane == 0) out[len] = found;
+        if (lane == 0) out[len] = nx;
         ++len;
-        cur = found;
+        cur = nx;
     }
     last = cur;
     return len;
