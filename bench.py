@@ -71,7 +71,7 @@ def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["jsv", "reference"], default="jsv")
     ap.add_argument("--workload", default="8b_64", choices=list(DESCRIPTION))
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -250,6 +250,13 @@ def accept_hist(accept_len):
     for a in accept_len:
         h[str(int(a))] = h.get(str(int(a)), 0) + 1
     return dict(sorted(h.items(), key=lambda kv: int(kv[0])))
+
+
+def tpf_mean(hist):
+    """Mean tokens per forward over the requests: accepted draft tokens plus
+    the bonus token, a + 1 (the accept-length histogram counts a)."""
+    n = sum(hist.values())
+    return sum((int(a) + 1) * c for a, c in hist.items()) / n if n else None
 
 
 def source_sha(*files):
@@ -504,7 +511,7 @@ def measure_workload(gb, name, K, warmup, pk):
            "step_hbm_bytes": model["step_hbm_bytes"], "step_flops": model["step_flops"],
            "call_us": {n: float(np.median(per[:, j]) * 1e3) for j, n in enumerate(CALLS)},
            "clocks": gb.clocks.summary([f"steps:{name}", f"calls:{name}"]),
-           "check": check, "accept_len_hist": hist}
+           "check": check, "accept_len_hist": hist, "tokens_per_forward_mean": tpf_mean(hist)}
     del st
     torch.cuda.empty_cache()
     return out
@@ -711,7 +718,7 @@ def run_gpu(args, rank, world, local_rank):
         "clocks": gb.clocks.summary(["steps", "calls", "graph"]),
         "clocks_all_regions": gb.clocks.summary(),
         "check": check,
-        "accept_len_hist": hist,
+        "accept_len_hist": hist, "tokens_per_forward_mean": tpf_mean(hist),
     }
     if qkv is not None:
         qkv["frac_of_hbm_peak"] = qkv["achieved_gbs"] / hbm
