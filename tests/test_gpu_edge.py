@@ -89,6 +89,12 @@ ATTN_CASES = {
     # 48 requests with prefixes from 16 to 1500 tokens and trees of 1 to 20
     # nodes: 384 (request, KV head) units, so the launch takes one split per
     # request and orders the units longest first
+    # no GQA packing at head dimension 128 (G = 1: 128 nodes per row group)
+    "g1_head_dim_128": ([synth.tiny_tree(np.random.default_rng(40), 150, 9, 3)], [300], 4, 4, 128),
+    # more requests than the longest-first order takes (70 > 64): block-index
+    # units, most of them single-tile requests, a few prefixes of zero
+    "b70_block_order": ([synth.tiny_tree(np.random.default_rng(500 + i), 1 + i % 5, 3, 2) for i in range(70)],
+                        [(37 * i) % 211 if i % 9 else 0 for i in range(70)], 4, 2, 64),
     "lpt_48_ragged": ([synth.tiny_tree(np.random.default_rng(300 + i), 1 + (7 * i) % 20, 4, 3) for i in range(48)],
                       [16 + (353 * i) % 1485 for i in range(48)], 16, 8, 64),
 }
