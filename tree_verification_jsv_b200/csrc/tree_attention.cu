@@ -13,9 +13,13 @@
 // start on page boundaries, followed by the tree tiles, which cover slots
 // [P & ~15, P + N) and apply the ancestor mask; split s takes a balanced
 // contiguous run of these tiles (a split that holds tree tiles builds the
-// ancestor bitsets).  Each split writes an unnormalised fp32
-// partial (O, row max, row sum); a small combine kernel merges the splits
-// with log-sum-exp rescaling and rounds to bf16.
+// ancestor bitsets).  A request takes as many splits as its tile count
+// needs at about C tiles each (at most S, the largest request's count).
+// Each split writes an unnormalised fp32 partial (O, row max, row sum); a
+// small combine kernel merges the splits with log-sum-exp rescaling and
+// rounds to bf16.  A request with one split writes its rows in bf16 from
+// this kernel, and the combine skips it.  When every request has one split
+// and the batch is small, the CTAs take the units longest first.
 //
 // Per CTA, 12 warps (three warpgroups):
 //   warp 0      TMA producer: Q once, then K and V of each 128-key tile, one
