@@ -40,6 +40,11 @@ CASES = {
     "ragged_300": ([synth.budget_tree(np.random.default_rng(3), n, 10, 4) for n in (100, 37, 163)],
                    [500, 1700, 33], 32, 8, 128, 1024),
     "g8_d2048": ([synth.budget_tree(np.random.default_rng(4), 96, 12, 8)], [777], 32, 4, 128, 2048),
+    # K splits of 4 (24 head tiles) and of 2 (64 head tiles), with node counts
+    # that leave a partial 32-node slice
+    "ksplit4_40_nodes": ([synth.budget_tree(np.random.default_rng(5), 40, 6, 4)], [300], 16, 4, 128, 1024),
+    "ksplit2_two_requests": ([synth.tiny_tree(np.random.default_rng(6), 29, 6, 3),
+                              synth.tiny_tree(np.random.default_rng(7), 21, 5, 3)], [90, 17], 48, 8, 128, 512),
 }
 
 
