@@ -104,7 +104,9 @@ typedef struct {
 } jsv_batch;
 
 /* Bytes of scratch jsv_tree_attention needs for this geometry (split-KV
- * partial results).  Depends only on the host-side fields. */
+ * partial results; 0 when every request takes one split).  Depends on the
+ * host-side fields and on the current device's SM count, which sets the
+ * split count. */
 JSV_API size_t jsv_tree_attention_workspace_size(const jsv_batch *batch);
 
 /*
@@ -120,6 +122,8 @@ JSV_API size_t jsv_tree_attention_workspace_size(const jsv_batch *batch);
  *   out      device [T][Hq][D] bf16
  *   workspace, workspace_bytes  device scratch of at least
  *            jsv_tree_attention_workspace_size(batch) bytes, 256-B aligned
+ *            (NULL is accepted when that size is 0); any contents, since
+ *            every call writes what it reads
  */
 JSV_API jsv_status jsv_tree_attention(const jsv_batch *batch, const uint16_t *q,
                               const uint16_t *k_cache, const uint16_t *v_cache,
