@@ -112,6 +112,31 @@ def test_attention_edge_cases(name, sharp):
     attention_close(got, run_oracle_attention(case), name)
 
 
+@pytest.mark.parametrize("seed", range(8))
+def test_attention_random_geometry(seed):
+    """Seeded random batches against the oracle: 1 to 70 requests (both unit
+    orders and both one and several splits), G in {1, 2, 3, 4, 8, 16}, D in
+    {64, 128}, prefixes from 0 to 2500 (page-aligned or not), trees of 1 to
+    180 nodes of random shape, and sharp queries in half of them."""
+    rng = np.random.default_rng(1000 + seed)
+    G = (1, 2, 3, 4, 8, 16, 4, 8)[seed]
+    B = (1, 2, 5, 17, 70, 3, 64, 1)[seed]
+    D = (64, 128)[(seed + seed // 4) % 2]
+    Hkv = int(rng.choice([1, 2])) if G >= 8 else int(rng.choice([1, 2, 4]))
+    cap = 180 if B <= 5 else 24
+    parents = []
+    for _ in range(B):
+        n = int(rng.integers(1, cap + 1))
+        depth = int(rng.integers(max(1, math.ceil(math.log2(n + 1))), 13))   # room for n nodes at 2+ children
+        parents.append(synth.tiny_tree(rng, n, depth, int(rng.integers(2, 5))))
+    pre = [int(rng.choice([0, 16, 17, 255, 1024, int(rng.integers(0, 2500))])) for _ in range(B)]
+    case = small_case(parents, pre, Hq=G * Hkv, Hkv=Hkv, D=D, seed=2000 + seed, q_scale=4.0 if seed % 2 else 1.0)
+    got, st = run_attention(case)
+    assert st == 0
+    from helpers import run_oracle_attention
+    attention_close(got, run_oracle_attention(case), f"random geometry {seed}")
+
+
 def test_attention_workspace_reused_without_clearing():
     """One attention workspace, filled with garbage once, serves calls of
     different batch shapes back to back on one stream: no call may depend on
