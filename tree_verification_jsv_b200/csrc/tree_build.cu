@@ -9,9 +9,11 @@
 //     score descending, depth ascending, rank path (lexicographic) ascending,
 // which is ancestor- and sibling-closed, emitted breadth-first.
 //
-// One CTA of 32 warps per request, no sorting and no heap:
-//  1. tau, the budget-th best score, by a 32-way search over the fp32 order
-//     (each round every warp tests one threshold, ~7 rounds instead of 32):
+// One CTA of 16 warps per request, no sorting and no heap:
+//  1. tau, the budget-th best score, by a 16-way search over the fp32 order
+//     (each round every warp tests one threshold, ~8 rounds instead of 32;
+//     a round costs one warp's expansion latency, so 16 warps measured
+//     faster than 32 or 8):
 //     count(x) = #nodes with score >= x comes from a level-by-level expansion
 //     that stops as soon as it reaches the budget (children of a node are
 //     scanned in rank order and stop at the first one below x, since the
@@ -60,7 +62,8 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
     return v;
 }
 
-constexpr int kTreeWarps = 32;                 // warps a request: one threshold each per round
+constexpr int kTreeWarpsLog2 = 4;
+constexpr int kTreeWarps = 1 << kTreeWarpsLog2;  // warps a request: one threshold each per round
 constexpr int kTreeLevel = kTreeMaxBudget + kTreeMaxWidth;
 
 struct TreeSmem {
@@ -162,16 +165,16 @@ accum_logp_tree_kernel(TreeArgs a) {
     if (search && !sm.take_all) {
         while (sm.hi - sm.lo > 1u) {
             const uint32_t lo = sm.lo, hi = sm.hi;
-            const uint32_t t = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)warp) >> 5);
+            const uint32_t t = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)warp) >> kTreeWarpsLog2);
             const int ok = warp == 0 ? 1 : (count_ge(sm, lvl0, lvl1, D, k, ord2f(t), budget, lane) >= budget);
             if (lane == 0) sm.res[warp] = ok;
             __syncthreads();
             if (threadIdx.x == 0) {
                 int w = kTreeWarps - 1;
                 while (w > 0 && !sm.res[w]) --w;
-                sm.lo = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)w) >> 5);
+                sm.lo = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)w) >> kTreeWarpsLog2);
                 if (w + 1 < kTreeWarps)
-                    sm.hi = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)(w + 1)) >> 5);
+                    sm.hi = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)(w + 1)) >> kTreeWarpsLog2);
             }
             __syncthreads();
         }
