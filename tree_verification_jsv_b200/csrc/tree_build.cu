@@ -79,30 +79,32 @@ struct TreeSmem {
 
 // Number of nodes with score >= x, capped at `cap` (exits as soon as it is
 // reached).  One warp, with its own two level buffers; the result is uniform.
+// Only the count and the set of next-level scores matter here (not their
+// order), so each 32-node chunk of a level is expanded one child rank at a
+// time with a ballot: a lane whose rank-r child falls below x has no later
+// passing child (the log-probs are sorted), and a rank that no lane passes
+// ends the chunk.
 __device__ int count_ge(const TreeSmem &sm, float *cur, float *nxt, int D, int k, float x, int cap, int lane) {
     if (lane == 0) cur[0] = 0.f;
     __syncwarp();
     int ncur = 1, total = 1;
     if (total >= cap) return cap;
+    const unsigned lt = (1u << lane) - 1u;
     for (int m = 0; m < D && ncur > 0; ++m) {
         int base = 0;
         for (int c0 = 0; c0 < ncur; c0 += 32) {
             const int i = c0 + lane;
-            float s = 0.f;
-            int cnt = 0;
-            if (i < ncur) {
-                s = cur[i];
-                for (int r = 0; r < k; ++r) {
-                    if (__fadd_rn(s, sm.lp[m][r]) >= x) ++cnt;
-                    else break;
-                }
+            const bool live = i < ncur;
+            const float s = live ? cur[i] : 0.f;
+            for (int r = 0; r < k; ++r) {
+                const float sc = __fadd_rn(s, sm.lp[m][r]);
+                const unsigned b = __ballot_sync(0xffffffffu, live && sc >= x);
+                if (b == 0u) break;
+                const int nb = __popc(b);
+                if (total + base + nb >= cap) return cap;
+                if ((b >> lane) & 1u) nxt[base + __popc(b & lt)] = sc;
+                base += nb;
             }
-            const int incl = warp_incl_scan(cnt, lane);
-            const int tot = __shfl_sync(0xffffffffu, incl, 31);
-            if (total + base + tot >= cap) return cap;
-            const int off = base + incl - cnt;
-            for (int r = 0; r < cnt; ++r) nxt[off + r] = __fadd_rn(s, sm.lp[m][r]);
-            base += tot;
         }
         __syncwarp();
         total += base;
