@@ -73,8 +73,9 @@ struct TreeSmem {
     uint8_t nrank[kTreeMaxBudget];
     uint8_t ndepth[kTreeMaxBudget];
     int res[kTreeWarps];
+    uint32_t tw[kTreeWarps];                   // the thresholds of a search round
     uint32_t lo, hi;
-    int bad, take_all, nodes;
+    int bad, take_all, nodes, vfirst;
 };
 
 // Number of nodes with score >= x, capped at `cap` (exits as soon as it is
@@ -149,13 +150,17 @@ accum_logp_tree_kernel(TreeArgs a) {
     }
 
     // 1. tau: the largest x with count(x) >= budget.  Invariant count(lo) >=
-    //    budget > count(hi) over the fp32 order; each round warp w tests
-    //    lo + (hi - lo) * w / 32 and the interval shrinks to the last passing
-    //    point and the next (count is non-increasing in x).
+    //    budget > count(hi) over the fp32 order; each round warp w tests a
+    //    threshold t_w (t_0 = lo, non-decreasing in w) and the interval
+    //    shrinks to the last passing threshold and the next (count is
+    //    non-increasing in x).  The first round spaces the thresholds evenly
+    //    in value over [smin, 0], where smin is the lowest score a node can
+    //    have; later rounds evenly over the fp32 order, lo + (hi - lo) w / W.
     if (threadIdx.x == 0) {
         sm.lo = f2ord(-INFINITY);
         sm.hi = f2ord(0.f) + 1u;
         sm.take_all = 0;
+        sm.vfirst = 0;
     }
     __syncthreads();
     const bool search = budget > 1 && D > 0;
@@ -165,18 +170,42 @@ accum_logp_tree_kernel(TreeArgs a) {
     }
     __syncthreads();
     if (search && !sm.take_all) {
+        // smin: every depth's smallest log-prob summed in fp32 in the order
+        // the expansion adds them; no node scores lower, so count(smin) is the
+        // whole candidate tree (at least the budget, as take_all is false)
+        if (threadIdx.x == 0) {
+            float smin = 0.f;
+            for (int m = 0; m < D; ++m) smin = __fadd_rn(smin, sm.lp[m][k - 1]);
+            if (smin > -INFINITY) {
+                sm.lo = f2ord(smin);
+                sm.vfirst = 1;
+            }
+        }
+        __syncthreads();
         while (sm.hi - sm.lo > 1u) {
             const uint32_t lo = sm.lo, hi = sm.hi;
-            const uint32_t t = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)warp) >> kTreeWarpsLog2);
+            uint32_t t;
+            if (sm.vfirst) {
+                const float v = ord2f(lo) * (1.f - (float)warp / (float)kTreeWarps);    // hi is just above 0
+                t = warp == 0 ? lo : min(max(f2ord(v), lo + 1u), hi - 1u);
+            } else {
+                t = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)warp) >> kTreeWarpsLog2);
+            }
             const int ok = warp == 0 ? 1 : (count_ge(sm, lvl0, lvl1, D, k, ord2f(t), budget, lane) >= budget);
-            if (lane == 0) sm.res[warp] = ok;
+            if (lane == 0) {
+                sm.res[warp] = ok;
+                sm.tw[warp] = t;
+            }
             __syncthreads();
-            if (threadIdx.x == 0) {
-                int w = kTreeWarps - 1;
-                while (w > 0 && !sm.res[w]) --w;
-                sm.lo = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)w) >> kTreeWarpsLog2);
-                if (w + 1 < kTreeWarps)
-                    sm.hi = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)(w + 1)) >> kTreeWarpsLog2);
+            if (warp == 0) {
+                // the last passing threshold (warp 0's, lo, always passes)
+                const unsigned pass = __ballot_sync(0xffffffffu, lane < kTreeWarps && sm.res[lane]);
+                const int w = 31 - __clz(pass);
+                if (lane == 0) {
+                    sm.lo = sm.tw[w];
+                    if (w + 1 < kTreeWarps) sm.hi = sm.tw[w + 1];
+                    sm.vfirst = 0;
+                }
             }
             __syncthreads();
         }
