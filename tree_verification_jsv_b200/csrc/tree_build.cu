@@ -53,15 +53,6 @@ __device__ __forceinline__ float ord2f(uint32_t o) {
     return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
-__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += t;
-    }
-    return v;
-}
-
 constexpr int kTreeWarpsLog2 = 4;
 constexpr int kTreeWarps = 1 << kTreeWarpsLog2;  // warps a request: one threshold each per round
 constexpr int kTreeLevel = kTreeMaxBudget + kTreeMaxWidth;
@@ -73,9 +64,10 @@ struct TreeSmem {
     uint8_t nrank[kTreeMaxBudget];
     uint8_t ndepth[kTreeMaxBudget];
     int res[kTreeWarps];
+    int cnt[kTreeWarps];                       // their counts (exact below the budget)
     uint32_t tw[kTreeWarps];                   // the thresholds of a search round
     uint32_t lo, hi;
-    int bad, take_all, nodes, vfirst;
+    int bad, take_all, nodes, vfirst, hi_count;
 };
 
 // Number of nodes with score >= x, capped at `cap` (exits as soon as it is
@@ -161,6 +153,7 @@ accum_logp_tree_kernel(TreeArgs a) {
         sm.hi = f2ord(0.f) + 1u;
         sm.take_all = 0;
         sm.vfirst = 0;
+        sm.hi_count = 0;                         // no node scores above 0
     }
     __syncthreads();
     const bool search = budget > 1 && D > 0;
@@ -191,9 +184,10 @@ accum_logp_tree_kernel(TreeArgs a) {
             } else {
                 t = lo + (uint32_t)(((unsigned long long)(hi - lo) * (unsigned)warp) >> kTreeWarpsLog2);
             }
-            const int ok = warp == 0 ? 1 : (count_ge(sm, lvl0, lvl1, D, k, ord2f(t), budget, lane) >= budget);
+            const int c = warp == 0 ? budget : count_ge(sm, lvl0, lvl1, D, k, ord2f(t), budget, lane);
             if (lane == 0) {
-                sm.res[warp] = ok;
+                sm.res[warp] = c >= budget;
+                sm.cnt[warp] = c;
                 sm.tw[warp] = t;
             }
             __syncthreads();
@@ -203,7 +197,10 @@ accum_logp_tree_kernel(TreeArgs a) {
                 const int w = 31 - __clz(pass);
                 if (lane == 0) {
                     sm.lo = sm.tw[w];
-                    if (w + 1 < kTreeWarps) sm.hi = sm.tw[w + 1];
+                    if (w + 1 < kTreeWarps) {
+                        sm.hi = sm.tw[w + 1];
+                        sm.hi_count = sm.cnt[w + 1];
+                    }
                     sm.vfirst = 0;
                 }
             }
@@ -228,9 +225,9 @@ accum_logp_tree_kernel(TreeArgs a) {
         } else if (!search) {
             ties_left = 0;
         } else {
-            const int n_gt = lo == f2ord(0.f) ? count_ge(sm, lvl0, lvl1, D, k, __uint_as_float(0x00000001u), budget, lane)
-                                              : count_ge(sm, lvl0, lvl1, D, k, ord2f(lo + 1u), budget, lane);
-            ties_left = budget - n_gt;
+            // the search ended at hi = lo + 1, a tested threshold whose count
+            // (below the budget, so exact) is the number of nodes above tau
+            ties_left = budget - sm.hi_count;
         }
         if (lane == 0) {
             sm.nscore[0] = 0.f;
@@ -243,26 +240,33 @@ accum_logp_tree_kernel(TreeArgs a) {
         for (int m = 0; m < D && lvl_begin < lvl_end && n < budget; ++m) {
             for (int c0 = lvl_begin; c0 < lvl_end; c0 += 32) {
                 const int i = c0 + lane;
-                float s = 0.f;
-                int cgt = 0, ceq = 0;
-                if (i < lvl_end) {
-                    s = sm.nscore[i];
-                    for (int r = 0; r < k; ++r) {
-                        const float cs = __fadd_rn(s, sm.lp[m][r]);
-                        if (cs > tau) ++cgt;
-                        else if (cs == tau) ++ceq;
-                        else break;
-                    }
+                const bool live = i < lvl_end;
+                const float s = live ? sm.nscore[i] : 0.f;
+                // a node's children above tau come first, then those equal to
+                // it (the log-probs are sorted); per rank, one ballot each for
+                // "above" and "equal" gives every lane its own counts and the
+                // counts of the lanes before it (a prefix sum without a scan)
+                const unsigned lt = (1u << lane) - 1u;
+                int cgt = 0, ceq = 0, pre_gt = 0, pre_eq = 0, tot_gt = 0, tot_eq = 0;
+                for (int r = 0; r < k; ++r) {
+                    const float cs = __fadd_rn(s, sm.lp[m][r]);
+                    const unsigned bg = __ballot_sync(0xffffffffu, live && cs > tau);
+                    const unsigned be = __ballot_sync(0xffffffffu, live && cs == tau);
+                    if ((bg | be) == 0u) break;
+                    cgt += (bg >> lane) & 1u;
+                    ceq += (be >> lane) & 1u;
+                    pre_gt += __popc(bg & lt);
+                    pre_eq += __popc(be & lt);
+                    tot_gt += __popc(bg);
+                    tot_eq += __popc(be);
                 }
-                // ties are taken in breadth-first order while the tie budget lasts
-                const int eq_incl = warp_incl_scan(ceq, lane);
-                const int eq_excl = eq_incl - ceq;
-                const int take_eq = max(0, min(ceq, ties_left - eq_excl));
+                // ties are taken in breadth-first order while the tie budget
+                // lasts: the lanes before this one took min(pre_eq, ties_left)
+                const int take_eq = max(0, min(ceq, ties_left - pre_eq));
                 const int c = cgt + take_eq;
-                const int incl = warp_incl_scan(c, lane);
-                const int tot = __shfl_sync(0xffffffffu, incl, 31);
-                const int used_eq = __shfl_sync(0xffffffffu, max(0, min(eq_incl, ties_left)), 31);
-                const int off = n + incl - c;
+                const int used_eq = min(tot_eq, ties_left);
+                const int tot = tot_gt + used_eq;
+                const int off = n + pre_gt + min(pre_eq, ties_left);
                 for (int r = 0; r < c && off + r < budget; ++r) {
                     sm.nscore[off + r] = __fadd_rn(s, sm.lp[m][r]);
                     sm.nparent[off + r] = i;
