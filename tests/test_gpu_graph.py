@@ -88,3 +88,52 @@ def test_host_step_matches_device_step(name):
         assert np.array_equal(outs[-1][k].numpy(), getattr(dev, k).cpu().numpy()), k
     for name_ in ("out", "argmax", "k_cache", "v_cache"):
         assert np.array_equal(_bits(getattr(dev, name_)), _bits(getattr(host, name_))), name_
+
+
+def _changed_tokens(wl, tokens, gold_arg):
+    """Draft tokens that the oracle accepts along other paths: every other
+    node's token moved off its value, and if that changes no path, node 1 of
+    each request given its parent's argmax (a match at depth 1)."""
+    import oracle
+    walk = lambda tok: oracle.accept_batch(wl.node_offsets, wl.parent, tok, gold_arg)
+    changed = np.where(np.arange(tokens.size) % 2 == 1, (tokens + 1) % wl.V, tokens).astype(np.int32)
+    if walk(changed) == walk(tokens):
+        for b in range(len(wl.node_offsets) - 1):
+            base = int(wl.node_offsets[b])
+            if int(wl.node_offsets[b + 1]) - base > 1:
+                changed[base + 1] = gold_arg[base + int(wl.parent[base + 1])]
+    assert walk(changed) != walk(tokens)
+    return changed
+
+
+@pytest.mark.parametrize("name", ["tiny", "8b_64"])
+def test_host_graph_matches_oracle(name):
+    """The end-to-end step from one CUDA graph (copy up, the calls, copy back)
+    matches the oracle, and its input copy reads the pinned arena when the
+    graph runs: draft tokens changed on the host between replays change the
+    accepted paths as the oracle says, and the returned host views equal the
+    device outputs."""
+    from tree_verification_jsv_b200 import build
+    from tree_verification_jsv_b200.step import VerifyStep
+    build.build()
+    wl, tokens, gold_arg = golden_workload(name)
+    k0, v0 = wl.k_cache.copy(), wl.v_cache.copy()
+    st = VerifyStep(wl, tokens)
+    kd, vd = st.k_cache.clone(), st.v_cache.clone()
+    st.capture_host()                       # runs one eager end-to-end step first
+    tokens = np.asarray(tokens, dtype=np.int32)
+    changed = _changed_tokens(wl, tokens, gold_arg)
+    for rep, tok in enumerate((tokens, changed, tokens)):
+        st.host_inputs()["tokens"].copy_(torch.from_numpy(tok))
+        st.k_cache.copy_(kd)
+        st.v_cache.copy_(vd)
+        st.status.zero_()
+        st.out.zero_()
+        st.argmax.fill_(-1)
+        st.path.fill_(-9)
+        torch.cuda.synchronize()
+        got = st.replay_host()
+        torch.cuda.synchronize()
+        assert_step_matches_oracle(st, wl, tok, gold_arg, k0, v0, f"{name} host replay {rep}")
+        for k in ("path", "accept_len", "bonus", "new_len"):
+            assert np.array_equal(got[k].numpy(), getattr(st, k).cpu().numpy()), (rep, k)

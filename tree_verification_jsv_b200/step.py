@@ -16,7 +16,9 @@ pinned host buffer, so each direction is a single copy.
 ``capture`` records the step's calls once into a CUDA graph (the engine the
 JetSpec README describes replays CUDA graphs for wall-clock latency); every
 kernel is launched with programmatic dependent launch, so the graph keeps
-those overlapping edges.  ``replay`` launches the whole step in one call.
+those overlapping edges.  ``replay`` launches the whole step in one call;
+``capture_host`` / ``replay_host`` do the same for the end-to-end form,
+copies included.
 """
 from __future__ import annotations
 
@@ -109,6 +111,7 @@ class VerifyStep:
         self.attn_ws = torch.zeros(max(aws, 256), dtype=torch.uint8, device=dev)   # any contents: every call writes what it reads
         self.lm_ws = torch.zeros(max(lws, 8), dtype=torch.uint8, device=dev)   # zeroed once; each call leaves it zeroed
         self._graph = None
+        self._host_graph = None
 
     # -- the four calls -----------------------------------------------------
     def attention(self, stream=None):
@@ -181,4 +184,28 @@ class VerifyStep:
         self._in.dev_buf.copy_(self._in.host_buf, non_blocking=True)
         self.run(stream)
         self._out.host_buf.copy_(self._out.dev_buf, non_blocking=True)
+        return self._out.host
+
+    def capture_host(self):
+        """Record the end-to-end step (the input arena's copy up from pinned
+        host memory, the step's calls, the output arena's copy back) into one
+        CUDA graph, so that ``replay_host`` issues all of it with one launch.
+        The graph's copies read and write the pinned buffers when it runs:
+        the caller fills ``host_inputs()`` before each replay and reads the
+        returned views after synchronising.  One eager ``run_host`` runs
+        first (one-time host set-up outside the capture)."""
+        self.run_host()
+        torch.cuda.synchronize(self.device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.run_host()
+        torch.cuda.synchronize(self.device)
+        self._host_graph = graph
+        return graph
+
+    def replay_host(self):
+        """One end-to-end step through the graph of ``capture_host``; returns
+        the pinned host views of path, accept_len, bonus and new_len (filled
+        once the current stream has been synchronised)."""
+        self._host_graph.replay()
         return self._out.host
