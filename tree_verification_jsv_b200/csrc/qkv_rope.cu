@@ -23,10 +23,12 @@
 // rows with 256 contiguous bytes).
 // When (tile, node group) CTAs alone would leave SMs idle (one 64-node tree:
 // 48 tiles for Qwen3-8B), a cluster of up to four CTAs splits K: each reduces
-// its share of d into its own TMEM, hands each 32-node slice of its partial
-// to the first CTA through distributed shared memory (bounded mbarrier
-// handshakes: ready on the first CTA, free on the others), and the first CTA
-// adds them and runs the epilogue.
+// its share of d into its own TMEM and stores each 32-node slice of its
+// partial into its own slot of the first CTA's shared memory (distributed
+// shared memory; bounded mbarrier handshakes: ready on the first CTA, free on
+// the others, the first free meaning that the first CTA's ring, which holds
+// the slots, is idle), and the first CTA adds the slots to its own partial
+// and runs the epilogue.
 // Under programmatic dependent launch the producer issues the first ring's
 // worth of W copies before it waits for the previous launch: W is a weight
 // that no call of this library writes, while x, the batch geometry and the
@@ -41,13 +43,20 @@ using namespace sm100;
 namespace {
 
 constexpr int kQThreads = 192;
-constexpr int kQMaxStages = 8;
+constexpr int kQMaxSplit = 4;                    // CTAs of a cluster splitting K
+constexpr int kQMaxStages = 6;
 constexpr int kQTileM = 128;
 constexpr int kQKChunk = 64;
 constexpr uint32_t kQStageA = kQTileM * 128;
-constexpr int kQSmemBudget = 164 * 1024;
+// The ring may take the shared memory the other arrays leave (the epilogue's
+// slice buffers reuse the ring once the accumulator is complete), up to six
+// stages: groups of 256 nodes (16 KB of W + 32 KB of x a stage) get four
+// stages instead of three, measured 50.0 -> 47.0 us for one 256-node tree of
+// Qwen3-8B shapes; more than six stages slowed the 64-node case (nine:
+// 26.8 -> 28.6 us), so the cap keeps it at six.
+constexpr int kQSmemBudget = 216 * 1024;
 // A smaller ring that lets two CTAs share an SM, so that clusters of three
-// find room in one resident wave (about 37 KB of static shared memory a CTA).
+// find room in one resident wave (about 5 KB of static shared memory a CTA).
 constexpr int kQSmemBudgetShared = 72 * 1024;
 constexpr int kQMaxWalk = 512 + 256;             // parents a group's depth walks can visit
 
@@ -66,7 +75,7 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float f) {
     return *reinterpret_cast<uint16_t *>(&h);
 }
 
-__global__ void __launch_bounds__(kQThreads, 1)
+__global__ void __launch_bounds__(kQThreads, 2)
 qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                 const QkvParams p) {
     pdl_allow_dependents();
@@ -75,14 +84,22 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ volatile int ep_fail;
+    // slice_ready (first CTA): the other CTAs' partials of a slice have
+    // landed; slice_free (other CTAs): the first CTA may take the next one
     __shared__ __align__(8) uint64_t slice_ready, slice_free;
-    __shared__ __align__(16) float tile[32][kQTileM];   // one 32-node slice, a row of 128 tile rows per node
-    __shared__ float xch[32][kQTileM];           // a K-split partial handed to the first CTA
     __shared__ int s_pos[256], s_row[256];
     __shared__ int s_par[kQMaxWalk];
 
     const BatchArgs &a = p.a;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+    // Epilogue buffers over the start of the ring, used once the first CTA's
+    // last MMA has completed (every stage consumed, no copy in flight): one
+    // 32-node slice, a row of 128 tile rows per node, then, in the first CTA,
+    // slot q for CTA q's partial of a slice (the same offsets in every CTA).
+    float (*tile)[kQTileM] = reinterpret_cast<float (*)[kQTileM]>(smem);
+    auto recv = [&](int q) {
+        return reinterpret_cast<float (*)[kQTileM]>(smem + (size_t)q * sizeof(float) * 32 * kQTileM);
+    };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // K split: CTA ks of the cluster reduces K-chunks [kc0, kc1); the first
     // CTA adds the others' partials and runs the epilogue
@@ -99,7 +116,7 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
         mbar_init(&accf_bar, 1);
         mbar_init(&drain_bar, 1);
-        mbar_init(&slice_ready, 4 * (p.ksplit > 1 ? p.ksplit - 1 : 1));  // the peers' epilogue warps
+        mbar_init(&slice_ready, 4 * (p.ksplit > 1 ? p.ksplit - 1 : 1));  // the other CTAs' epilogue warps
         mbar_init(&slice_free, 4);                                       // the first CTA's epilogue warps
         abort_sh = 0;
         ep_fail = 0;
@@ -244,6 +261,19 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         named_barrier(1, 128);
 
         const int qrows = a.Hq * a.D, krows = a.Hkv * a.D, half = a.D / 2;
+        // While the main loop runs, the rotary tables' rows at this group's
+        // positions go to L2 (only the first CTA of a cluster rotates, and
+        // only tiles with Q or K rows).
+        if (ks == 0 && row0 < qrows + krows) {
+            for (int c = et; c < in_group; c += 128) {
+                const int pos = s_pos[c];
+                if (pos < 0 || pos >= p.max_pos) continue;
+                for (int off = 0; off < half; off += 32) {          // 128-byte lines
+                    prefetch_l2(p.cos + (size_t)pos * half + off);
+                    prefetch_l2(p.sin + (size_t)pos * half + off);
+                }
+            }
+        }
 
         if (!mbar_wait(&accf_bar, 0, &abort_sh)) {
             abort_sh = 1;
@@ -253,58 +283,25 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         named_barrier(1, 128);
         if (!ep_fail) {
             tc_fence_after();
+            // The first CTA's ring is idle from here on: the other CTAs may
+            // store their first slice into its slots (the first phase of their
+            // slice_free).
+            if (ks == 0 && p.ksplit > 1 && lane == 0)
+                for (int q = 1; q < p.ksplit; ++q) mbar_arrive_cluster(cluster_addr(&slice_free, (uint32_t)q));
+            // Each warp takes 8 of a slice's 32 nodes (x = sub + 4k) and each
+            // lane 4 consecutive rows of the tile, so a warp writes a node's
+            // 128 rows as 256 contiguous bytes with one 8-byte store a lane.
+            const int q0 = lane * 4;                        // tile rows q0 .. q0 + 3
+            const int g0 = row0 + q0;
+            const int kq = g0 < qrows ? 0 : (g0 < qrows + krows ? 1 : 2);   // Q, K, V
+            const int hq = kq == 0 ? g0 : (kq == 1 ? g0 - qrows : g0 - qrows - krows);
+            const int headq = hq / a.D, oq = hq % a.D, iq = oq % half;
+            const bool qvalid = g0 + 3 < p.rows_total;
             for (int c0 = 0, sl = 0; c0 < in_group; c0 += 32, ++sl) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)c0, v);
-                tmem_ld_wait();
-                if (ks > 0) {
-                    // hand this slice to the first CTA (once it has taken the previous one)
-                    bool okw = sl == 0 || mbar_wait_cluster(&slice_free, (uint32_t)((sl - 1) & 1), &abort_sh);
-                    if (__any_sync(0xffffffffu, !okw)) {
-                        if (lane == 0) flag_error(a.dev_status, JSV_ERR_TIMEOUT);
-                        break;
-                    }
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) xch[x][r] = __uint_as_float(v[x]);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&slice_ready, 0));
-                    continue;
-                }
-                if (p.ksplit > 1) {
-                    // add the other CTAs' partials of this slice, then release them
-                    bool okw = mbar_wait_cluster(&slice_ready, (uint32_t)(sl & 1), &abort_sh);
-                    if (__any_sync(0xffffffffu, !okw)) {
-                        if (lane == 0) flag_error(a.dev_status, JSV_ERR_TIMEOUT);
-                        break;
-                    }
-                    for (int q = 1; q < p.ksplit; ++q) {
-                        // all 32 remote loads in flight before the first add
-                        const uint32_t base = cluster_addr(&xch[0][r], (uint32_t)q);
-                        float pq[32];
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) pq[x] = ld_shared_cluster_f32(base + (uint32_t)(x * kQTileM * 4));
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) + pq[x]);
-                    }
-                    __syncwarp();
-                    if (lane == 0)
-                        for (int q = 1; q < p.ksplit; ++q) mbar_arrive_cluster(cluster_addr(&slice_free, (uint32_t)q));
-                }
-#pragma unroll
-                for (int x = 0; x < 32; ++x) tile[x][r] = __uint_as_float(v[x]);
-                named_barrier(1, 128);
-                // Each warp takes 8 of the slice's 32 nodes (x = sub + 4k) and each
-                // lane 4 consecutive rows of the tile, so a warp writes a node's
-                // 128 rows as 256 contiguous bytes with one 8-byte store a lane.
-                // The slice's cos/sin loads are all issued before any is used.
-                {
-                    const int q0 = lane * 4;                        // tile rows q0 .. q0 + 3
-                    const int g0 = row0 + q0;
-                    const int kq = g0 < qrows ? 0 : (g0 < qrows + krows ? 1 : 2);   // Q, K, V
-                    const int hq = kq == 0 ? g0 : (kq == 1 ? g0 - qrows : g0 - qrows - krows);
-                    const int headq = hq / a.D, oq = hq % a.D, iq = oq % half;
-                    const bool qvalid = g0 + 3 < p.rows_total;
-                    float4 cs[8], sn[8];
+                // the slice's cos/sin loads go out first, so their latency
+                // overlaps the accumulator read and the cross-CTA sum
+                float4 cs[8], sn[8];
+                if (ks == 0) {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int c = c0 + sub + 4 * k;
@@ -313,10 +310,56 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         sn[k] = make_float4(0.f, 0.f, 0.f, 0.f);
                         if (kq < 2 && qvalid && pos >= 0 &&
                             JSV_IN_BOUNDS((long long)pos * half + iq + 3, (long long)p.max_pos * half, a.dev_status)) {
-                            cs[k] = __ldg(reinterpret_cast<const float4 *>(p.cos + (size_t)pos * half + iq));
-                            sn[k] = __ldg(reinterpret_cast<const float4 *>(p.sin + (size_t)pos * half + iq));
+                            cs[k] = ld_global_nc_f4(p.cos + (size_t)pos * half + iq);
+                            sn[k] = ld_global_nc_f4(p.sin + (size_t)pos * half + iq);
                         }
                     }
+                }
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)c0, v);
+                tmem_ld_wait();
+                if (ks > 0) {
+                    // store this partial into the first CTA's slot once the slot is
+                    // free (for the first slice: once the first CTA's ring is idle);
+                    // the first CTA reads it locally.  A warp whose wait runs out
+                    // (in any lane) skips its stores and goes on (no named barrier
+                    // on this path).
+                    if (!__all_sync(0xffffffffu, mbar_wait_cluster(&slice_free, (uint32_t)(sl & 1), &abort_sh))) {
+                        if (lane == 0) flag_error(a.dev_status, JSV_ERR_TIMEOUT);
+                        continue;
+                    }
+                    const uint32_t dst = cluster_addr(&recv(ks)[0][r], 0);
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) st_shared_cluster_b32(dst + (uint32_t)(x * kQTileM * 4), v[x]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&slice_ready, 0));
+                    continue;
+                }
+                if (p.ksplit > 1) {
+                    // add the other CTAs' partials of this slice in rank (K) order,
+                    // then release the slots.  A warp whose wait runs out raises
+                    // ep_fail and still takes the slice's named barriers; every
+                    // warp then leaves after the first of them.
+                    if (__all_sync(0xffffffffu, mbar_wait_cluster(&slice_ready, (uint32_t)(sl & 1), &abort_sh))) {
+                        for (int q = 1; q < p.ksplit; ++q) {
+                            const float(*pq)[kQTileM] = recv(q);
+#pragma unroll
+                            for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) + pq[x][r]);
+                        }
+                        __syncwarp();
+                        if (lane == 0)
+                            for (int q = 1; q < p.ksplit; ++q)
+                                mbar_arrive_cluster(cluster_addr(&slice_free, (uint32_t)q));
+                    } else if (lane == 0) {
+                        flag_error(a.dev_status, JSV_ERR_TIMEOUT);
+                        ep_fail = 1;
+                    }
+                }
+#pragma unroll
+                for (int x = 0; x < 32; ++x) tile[x][r] = __uint_as_float(v[x]);
+                named_barrier(1, 128);
+                if (ep_fail) break;                         // every epilogue warp sees the same flag here
+                {
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const int x = sub + 4 * k, c = c0 + x;
@@ -375,6 +418,7 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
     p.stage_bytes = kQStageA + (uint32_t)p.box_rows * 128;
     auto stages_for = [&](int budget) { return min(kQMaxStages, budget / (int)p.stage_bytes); };
     p.stages = stages_for(kQSmemBudget);
+    if ((size_t)p.stages * p.stage_bytes < 2 * 32 * kQTileM * sizeof(float)) return cudaErrorInvalidValue;
     p.cos = rope_cos;
     p.sin = rope_sin;
     p.max_pos = max_pos;
@@ -409,12 +453,13 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
     // SM; more CTAs streaming W beat a deeper ring per CTA.
     const int sms = device_sm_count();
     int ks = 1;
-    while (ks < 4 && (long long)tiles * groups * (ks + 1) <= sms && p.kchunks / (ks + 1) >= 4) ++ks;
+    while (ks < kQMaxSplit && (long long)tiles * groups * (ks + 1) <= sms && p.kchunks / (ks + 1) >= 4) ++ks;
     bool placed = false;
     for (; ks > 1 && !placed; --ks) {
         for (int budget : {kQSmemBudget, kQSmemBudgetShared}) {
             const int st_n = stages_for(budget);
-            if (st_n < 2) continue;
+            // the ring holds the slice buffer and a slot per other CTA
+            if (st_n < 2 || (size_t)st_n * p.stage_bytes < (size_t)ks * 32 * kQTileM * sizeof(float)) continue;
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(tiles * ks, groups);
             cfg.blockDim = dim3(kQThreads);
