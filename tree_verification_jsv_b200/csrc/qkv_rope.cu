@@ -70,6 +70,26 @@ struct QkvParams {
     uint16_t *q, *k_cache, *v_cache;
 };
 
+// Hint: bring the 128-byte line holding global address p into L2.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
+// Store to a shared::cluster address (from cluster_addr).
+__device__ __forceinline__ void st_shared_cluster_b32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// 16-byte read-only global load issued where it stands (not moved by the
+// compiler), so that its latency overlaps the code that follows.
+__device__ __forceinline__ float4 ld_global_nc_f4(const float *p) {
+    float4 v;
+    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(reinterpret_cast<uint64_t>(p)));
+    return v;
+}
+
 __device__ __forceinline__ uint16_t to_bf16_bits(float f) {
     __nv_bfloat16 h = __float2bfloat16_rn(f);
     return *reinterpret_cast<uint16_t *>(&h);

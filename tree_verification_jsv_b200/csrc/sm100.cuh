@@ -123,10 +123,6 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     return p;
 }
 
-// Hint: bring the 128-byte line holding global address p into L2.
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
-}
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -309,6 +305,13 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
         if (globaltimer() - t0 > limit_ns) return false;
     }
 }
+// Ordered after earlier volatile asm (the barrier wait that publishes the
+// data) but with no memory clobber, so a run of these stays in flight together.
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr));
+    return v;
+}
 // Complete `bytes` of the current phase's expected transaction count without
 // a copy (used when unwinding, for copies that were never issued).
 __device__ __forceinline__ void mbar_complete_tx(uint64_t *bar, uint32_t bytes) {
@@ -317,19 +320,6 @@ __device__ __forceinline__ void mbar_complete_tx(uint64_t *bar, uint32_t bytes) 
 // Store to a 32-bit shared variable of CTA `rank` of the cluster.
 __device__ __forceinline__ void st_shared_cluster_u32(const void *p, uint32_t rank, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr(p, rank)), "r"(v) : "memory");
-}
-// Store to a shared::cluster address (from cluster_addr).
-__device__ __forceinline__ void st_shared_cluster_b32(uint32_t cluster_addr, uint32_t v) {
-    asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-// 16-byte read-only global load issued where it stands (not moved by the
-// compiler), so that its latency overlaps the code that follows.
-__device__ __forceinline__ float4 ld_global_nc_f4(const float *p) {
-    float4 v;
-    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "l"(reinterpret_cast<uint64_t>(p)));
-    return v;
 }
 __device__ __forceinline__ uint32_t ld_shared_cluster_u32(const void *p, uint32_t rank) {
     uint32_t v;
