@@ -49,7 +49,8 @@ constexpr int kQTileM = 128;
 constexpr int kQKChunk = 64;
 constexpr uint32_t kQStageA = kQTileM * 128;
 // The ring may take the shared memory the other arrays leave (the epilogue's
-// slice buffers reuse the ring once the accumulator is complete), up to six
+// slice buffer and the K-split slots reuse the ring once the accumulator is
+// complete), up to six
 // stages: groups of 256 nodes (16 KB of W + 32 KB of x a stage) get four
 // stages instead of three, measured 50.0 -> 47.0 us for one 256-node tree of
 // Qwen3-8B shapes; more than six stages slowed the 64-node case (nine:
