@@ -45,6 +45,9 @@ CASES = {
     "ksplit4_40_nodes": ([synth.budget_tree(np.random.default_rng(5), 40, 6, 4)], [300], 16, 4, 128, 1024),
     "ksplit2_two_requests": ([synth.tiny_tree(np.random.default_rng(6), 29, 6, 3),
                               synth.tiny_tree(np.random.default_rng(7), 21, 5, 3)], [90, 17], 48, 8, 128, 512),
+    # one 256-node tree of Qwen3-8B shapes: a K split of 2 whose eight 32-node
+    # slices pass through the first CTA's slots (handshake phases wrap)
+    "qwen3_8b_256": ([synth.budget_tree(np.random.default_rng(9), 256, 16, 8)], [4000], 32, 8, 128, 4096),
 }
 
 
