@@ -23,12 +23,12 @@
 // rows with 256 contiguous bytes).
 // When (tile, node group) CTAs alone would leave SMs idle (one 64-node tree:
 // 48 tiles for Qwen3-8B), a cluster of up to four CTAs splits K: each reduces
-// its share of d into its own TMEM and stores each 32-node slice of its
-// partial into its own slot of the first CTA's shared memory (distributed
-// shared memory; bounded mbarrier handshakes: ready on the first CTA, free on
-// the others, the first free meaning that the first CTA's ring, which holds
-// the slots, is idle), and the first CTA adds the slots to its own partial
-// and runs the epilogue.
+// its share of d into its own TMEM and, once the first CTA's ring is idle,
+// stores every 32-node slice of its partial into a slot of its own in the
+// first CTA's shared memory (distributed shared memory; bounded mbarrier
+// handshakes: ring idle on the others, one ready per slice on the first CTA),
+// and the first CTA adds the slots to its own partial slice by slice and runs
+// the epilogue.
 // Under programmatic dependent launch the producer issues the first ring's
 // worth of W copies before it waits for the previous launch: W is a weight
 // that no call of this library writes, while x, the batch geometry and the
@@ -44,6 +44,7 @@ namespace {
 
 constexpr int kQThreads = 192;
 constexpr int kQMaxSplit = 4;                    // CTAs of a cluster splitting K
+constexpr int kQMaxSlices = 8;                   // 32-node slices of a group (at most 256 nodes)
 constexpr int kQMaxStages = 6;
 constexpr int kQTileM = 128;
 constexpr int kQKChunk = 64;
@@ -105,9 +106,10 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ volatile int ep_fail;
-    // slice_ready (first CTA): the other CTAs' partials of a slice have
-    // landed; slice_free (other CTAs): the first CTA may take the next one
-    __shared__ __align__(8) uint64_t slice_ready, slice_free;
+    // slice_ready[sl] (first CTA): the other CTAs' partials of slice sl have
+    // landed; ring_idle (other CTAs): the first CTA's ring, which holds the
+    // slots, is idle.  One phase each.
+    __shared__ __align__(8) uint64_t slice_ready[kQMaxSlices], ring_idle;
     __shared__ int s_pos[256], s_row[256];
     __shared__ int s_par[kQMaxWalk];
 
@@ -116,10 +118,14 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     // Epilogue buffers over the start of the ring, used once the first CTA's
     // last MMA has completed (every stage consumed, no copy in flight): one
     // 32-node slice, a row of 128 tile rows per node, then, in the first CTA,
-    // slot q for CTA q's partial of a slice (the same offsets in every CTA).
+    // a slot for every (other CTA q, slice) pair (the same offsets in every
+    // CTA), so the other CTAs store all their slices as soon as the ring is
+    // idle (the launch only splits K where the ring has room for them).
     float (*tile)[kQTileM] = reinterpret_cast<float (*)[kQTileM]>(smem);
-    auto recv = [&](int q) {
-        return reinterpret_cast<float (*)[kQTileM]>(smem + (size_t)q * sizeof(float) * 32 * kQTileM);
+    const int nslices = (p.group_nodes + 31) / 32;
+    auto recv = [&](int q, int sl) {
+        return reinterpret_cast<float (*)[kQTileM]>(smem + (size_t)(1 + (q - 1) * nslices + sl) * sizeof(float) * 32 *
+                                                              kQTileM);
     };
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // K split: CTA ks of the cluster reduces K-chunks [kc0, kc1); the first
@@ -137,8 +143,9 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         }
         mbar_init(&accf_bar, 1);
         mbar_init(&drain_bar, 1);
-        mbar_init(&slice_ready, 4 * (p.ksplit > 1 ? p.ksplit - 1 : 1));  // the other CTAs' epilogue warps
-        mbar_init(&slice_free, 4);                                       // the first CTA's epilogue warps
+        for (int sl = 0; sl < kQMaxSlices; ++sl)                         // the other CTAs' epilogue warps
+            mbar_init(&slice_ready[sl], 4 * (p.ksplit > 1 ? p.ksplit - 1 : 1));
+        mbar_init(&ring_idle, 4);                                        // the first CTA's epilogue warps
         abort_sh = 0;
         ep_fail = 0;
         fence_barrier_init();
@@ -305,10 +312,9 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
         if (!ep_fail) {
             tc_fence_after();
             // The first CTA's ring is idle from here on: the other CTAs may
-            // store their first slice into its slots (the first phase of their
-            // slice_free).
+            // store their partials into its slots.
             if (ks == 0 && p.ksplit > 1 && lane == 0)
-                for (int q = 1; q < p.ksplit; ++q) mbar_arrive_cluster(cluster_addr(&slice_free, (uint32_t)q));
+                for (int q = 1; q < p.ksplit; ++q) mbar_arrive_cluster(cluster_addr(&ring_idle, (uint32_t)q));
             // Each warp takes 8 of a slice's 32 nodes (x = sub + 4k) and each
             // lane 4 consecutive rows of the tile, so a warp writes a node's
             // 128 rows as 256 contiguous bytes with one 8-byte store a lane.
@@ -318,6 +324,7 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
             const int hq = kq == 0 ? g0 : (kq == 1 ? g0 - qrows : g0 - qrows - krows);
             const int headq = hq / a.D, oq = hq % a.D, iq = oq % half;
             const bool qvalid = g0 + 3 < p.rows_total;
+            bool ring_ok = false;                   // (other CTAs) the first CTA's ring was seen idle
             for (int c0 = 0, sl = 0; c0 < in_group; c0 += 32, ++sl) {
                 // the slice's cos/sin loads go out first, so their latency
                 // overlaps the accumulator read and the cross-CTA sum
@@ -340,37 +347,34 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 tmem_ld_32x32b_x32(tmem + lane_addr + (uint32_t)c0, v);
                 tmem_ld_wait();
                 if (ks > 0) {
-                    // store this partial into the first CTA's slot once the slot is
-                    // free (for the first slice: once the first CTA's ring is idle);
-                    // the first CTA reads it locally.  A warp whose wait runs out
-                    // (in any lane) skips its stores and goes on (no named barrier
-                    // on this path).
-                    if (!__all_sync(0xffffffffu, mbar_wait_cluster(&slice_free, (uint32_t)(sl & 1), &abort_sh))) {
+                    // store this partial into its slot of the first CTA once that
+                    // CTA's ring is idle (waited for before the first slice); the
+                    // first CTA reads it locally.  A warp whose wait runs out (in
+                    // any lane) skips its stores from then on (no named barrier on
+                    // this path).
+                    if (sl == 0) ring_ok = __all_sync(0xffffffffu, mbar_wait_cluster(&ring_idle, 0u, &abort_sh));
+                    if (!ring_ok) {
                         if (lane == 0) flag_error(a.dev_status, JSV_ERR_TIMEOUT);
                         continue;
                     }
-                    const uint32_t dst = cluster_addr(&recv(ks)[0][r], 0);
+                    const uint32_t dst = cluster_addr(&recv(ks, sl)[0][r], 0);
 #pragma unroll
                     for (int x = 0; x < 32; ++x) st_shared_cluster_b32(dst + (uint32_t)(x * kQTileM * 4), v[x]);
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&slice_ready, 0));
+                    if (lane == 0) mbar_arrive_cluster(cluster_addr(&slice_ready[sl], 0));
                     continue;
                 }
                 if (p.ksplit > 1) {
-                    // add the other CTAs' partials of this slice in rank (K) order,
-                    // then release the slots.  A warp whose wait runs out raises
-                    // ep_fail and still takes the slice's named barriers; every
-                    // warp then leaves after the first of them.
-                    if (__all_sync(0xffffffffu, mbar_wait_cluster(&slice_ready, (uint32_t)(sl & 1), &abort_sh))) {
+                    // add the other CTAs' partials of this slice in rank (K) order.
+                    // A warp whose wait runs out raises ep_fail and still takes the
+                    // slice's named barriers; every warp then leaves after the
+                    // first of them.
+                    if (__all_sync(0xffffffffu, mbar_wait_cluster(&slice_ready[sl], 0u, &abort_sh))) {
                         for (int q = 1; q < p.ksplit; ++q) {
-                            const float(*pq)[kQTileM] = recv(q);
+                            const float(*pq)[kQTileM] = recv(q, sl);
 #pragma unroll
                             for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) + pq[x][r]);
                         }
-                        __syncwarp();
-                        if (lane == 0)
-                            for (int q = 1; q < p.ksplit; ++q)
-                                mbar_arrive_cluster(cluster_addr(&slice_free, (uint32_t)q));
                     } else if (lane == 0) {
                         flag_error(a.dev_status, JSV_ERR_TIMEOUT);
                         ep_fail = 1;
@@ -479,8 +483,9 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
     for (; ks > 1 && !placed; --ks) {
         for (int budget : {kQSmemBudget, kQSmemBudgetShared}) {
             const int st_n = stages_for(budget);
-            // the ring holds the slice buffer and a slot per other CTA
-            if (st_n < 2 || (size_t)st_n * p.stage_bytes < (size_t)ks * 32 * kQTileM * sizeof(float)) continue;
+            // the ring holds the slice buffer and a slot per (other CTA, slice)
+            const size_t slots = 1 + (size_t)(ks - 1) * ((p.group_nodes + 31) / 32);
+            if (st_n < 2 || (size_t)st_n * p.stage_bytes < slots * 32 * kQTileM * sizeof(float)) continue;
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(tiles * ks, groups);
             cfg.blockDim = dim3(kQThreads);
