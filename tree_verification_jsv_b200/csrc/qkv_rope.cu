@@ -36,6 +36,10 @@
 #include "jsv_internal.cuh"
 #include "sm100.cuh"
 
+#include <map>
+#include <mutex>
+#include <tuple>
+
 namespace jsv {
 
 using namespace sm100;
@@ -428,6 +432,31 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
     }
 }
 
+// Clusters of `cfg` that fit on the current device at once, remembered per
+// (device, cluster size, dynamic shared memory): the occupancy query costs
+// host time that every call would otherwise pay.  Failed queries are not
+// remembered.
+int active_clusters(cudaLaunchConfig_t &cfg, int ks) {
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, size_t>, int> known;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const auto key = std::make_tuple(dev, ks, cfg.dynamicSmemBytes);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        const auto it = known.find(key);
+        if (it != known.end()) return it->second;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, qkv_rope_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    known[key] = n;
+    return n;
+}
+
 }  // namespace
 
 cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const uint16_t *w_qkv, int d,
@@ -497,11 +526,7 @@ cudaError_t launch_tree_qkv_rope(const BatchArgs &a, const uint16_t *x, const ui
             attr[0].val.clusterDim.z = 1;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, qkv_rope_kernel, &cfg) != cudaSuccess) {
-                cudaGetLastError();
-                n = 0;
-            }
+            const int n = active_clusters(cfg, ks);
             if ((long long)n >= (long long)tiles * groups) {     // one resident wave
                 p.stages = st_n;
                 smem = cfg.dynamicSmemBytes;
