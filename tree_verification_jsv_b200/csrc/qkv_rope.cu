@@ -388,33 +388,43 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                 for (int x = 0; x < 32; ++x) tile[x][r] = __uint_as_float(v[x]);
                 named_barrier(1, 128);
                 if (ep_fail) break;                         // every epilogue warp sees the same flag here
-                {
+                // One epilogue warp per SM sub-partition, so nothing hides a
+                // dependent chain: every read of a half-slice goes out before any
+                // use, and only the stores are predicated.
+                const float sg = oq < half ? -1.f : 1.f;             // rotate-half sign
+                uint16_t *const base = kq == 0 ? p.q : (kq == 1 ? p.k_cache : p.v_cache);
+                const long long dn = kq == 0 ? (long long)a.total_nodes * a.Hq * a.D
+                                             : (long long)a.num_pages * a.page_size * a.Hkv * a.D;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int x = sub + 4 * k, c = c0 + x;
-                        if (c >= in_group || !qvalid) continue;
-                        const int pos = s_pos[c], prow = s_row[c];
-                        if (pos < 0 || prow < 0) continue;
-                        float4 v = *reinterpret_cast<const float4 *>(&tile[x][q0]);
+                for (int h4 = 0; h4 < 8; h4 += 4) {
+                    int row_of[4];
+                    float4 vv[4], pp[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int x = sub + 4 * (h4 + k), c = c0 + x;
+                        const bool ok = qvalid && c < in_group && s_pos[c] >= 0 && s_row[c] >= 0;
+                        row_of[k] = !ok ? -1 : (kq == 0 ? node0 + c : s_row[c]);
+                        vv[k] = *reinterpret_cast<const float4 *>(&tile[x][q0]);
+                        pp[k] = *reinterpret_cast<const float4 *>(&tile[x][q0 ^ half]);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        float4 v = vv[k];
                         if (kq < 2) {
-                            const float4 pv = *reinterpret_cast<const float4 *>(&tile[x][q0 ^ half]);
-                            const float sg = oq < half ? -1.f : 1.f;     // rotate-half sign
-                            v.x = fmaf(v.x, cs[k].x, sg * pv.x * sn[k].x);
-                            v.y = fmaf(v.y, cs[k].y, sg * pv.y * sn[k].y);
-                            v.z = fmaf(v.z, cs[k].z, sg * pv.z * sn[k].z);
-                            v.w = fmaf(v.w, cs[k].w, sg * pv.w * sn[k].w);
+                            const float4 c4 = cs[h4 + k], s4 = sn[h4 + k], pv = pp[k];
+                            v.x = fmaf(v.x, c4.x, sg * pv.x * s4.x);
+                            v.y = fmaf(v.y, c4.y, sg * pv.y * s4.y);
+                            v.z = fmaf(v.z, c4.z, sg * pv.z * s4.z);
+                            v.w = fmaf(v.w, c4.w, sg * pv.w * s4.w);
                         }
+                        if (row_of[k] < 0) continue;
                         uint2 pk;
                         pk.x = (uint32_t)to_bf16_bits(v.x) | ((uint32_t)to_bf16_bits(v.y) << 16);
                         pk.y = (uint32_t)to_bf16_bits(v.z) | ((uint32_t)to_bf16_bits(v.w) << 16);
-                        const int t = node0 + c;
-                        const long long di = kq == 0 ? ((long long)t * a.Hq + headq) * a.D + oq
-                                                     : ((long long)prow * a.Hkv + headq) * a.D + oq;
-                        const long long dn = kq == 0 ? (long long)a.total_nodes * a.Hq * a.D
-                                                     : (long long)a.num_pages * a.page_size * a.Hkv * a.D;
+                        // q row: the node; cache row: its physical slot
+                        const long long di = ((long long)row_of[k] * (kq == 0 ? a.Hq : a.Hkv) + headq) * a.D + oq;
                         if (!JSV_IN_BOUNDS(di + 3, dn, a.dev_status)) continue;
-                        uint16_t *dst = (kq == 0 ? p.q : (kq == 1 ? p.k_cache : p.v_cache)) + di;
-                        *reinterpret_cast<uint2 *>(dst) = pk;
+                        *reinterpret_cast<uint2 *>(base + di) = pk;
                     }
                 }
                 named_barrier(1, 128);
