@@ -96,9 +96,11 @@ __device__ __forceinline__ float4 ld_global_nc_f4(const float *p) {
     return v;
 }
 
-__device__ __forceinline__ uint16_t to_bf16_bits(float f) {
-    __nv_bfloat16 h = __float2bfloat16_rn(f);
-    return *reinterpret_cast<uint16_t *>(&h);
+// Two floats rounded to nearest-even bf16 with one packed conversion; lo in
+// the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
 }
 
 __global__ void __launch_bounds__(kQThreads, 2)
@@ -419,8 +421,8 @@ qkv_rope_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__
                         }
                         if (row_of[k] < 0) continue;
                         uint2 pk;
-                        pk.x = (uint32_t)to_bf16_bits(v.x) | ((uint32_t)to_bf16_bits(v.y) << 16);
-                        pk.y = (uint32_t)to_bf16_bits(v.z) | ((uint32_t)to_bf16_bits(v.w) << 16);
+                        pk.x = pack_bf16x2_rn(v.x, v.y);
+                        pk.y = pack_bf16x2_rn(v.z, v.w);
                         // q row: the node; cache row: its physical slot
                         const long long di = ((long long)row_of[k] * (kq == 0 ? a.Hq : a.Hkv) + headq) * a.D + oq;
                         if (!JSV_IN_BOUNDS(di + 3, dn, a.dev_status)) continue;
